@@ -1,0 +1,420 @@
+"""Benchmark of one tree-verify step on B200: prints ONE JSON line (rank 0).
+
+A step is the whole hot path over one batch: tree_prepare -> tree_verify_attn (+ split merge)
+-> acceptance (greedy tree, or chain rejection sampling) -> kv_commit.  Metric: verified tree
+tokens per second (sum of tree nodes over the timed steps / device time), with the attention
+call's achieved HBM bandwidth against the measured copy bandwidth as the roofline figure.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload tree26] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank verifies its own batch (its own seeded sequences), no
+collective on the data path; the timed region is bracketed by a barrier and a synchronize, the
+time is the max over ranks, value = tokens of all ranks / that time ("weak" scaling).
+`--impl reference` times the fp64 CPU oracle on host cores on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+DEFAULT_WORKLOAD = "tree26"
+DESCR = {
+    "tiny": "B=1 Hq=8 Hkv=2 d=64 fp32, L=128, 8-node tree, V=256",
+    "tree26": "Llama-3-8B-shaped verify: B=1 Hq=32 Hkv=8 d=128 bf16, L=2048, static EAGLE tree N=26 "
+              "(4,3,2,1,1,1), V=128256, greedy, contiguous cache",
+    "eagle60": "B=16 Hq=32 Hkv=8 d=128 bf16, ragged L in [1024,8192], EAGLE-2 trees N=60, V=128256, "
+               "greedy, paged cache (block 16)",
+    "chain5": "70B-shaped chain: B=64 Hq=64 Hkv=8 d=128 bf16, L=8192, K=5, T=1 rejection sampling, V=128256",
+    "forest": "SSD forest: B=8 x 8 subtrees x 64 nodes, L=32768, Hq=32 Hkv=8 d=128 bf16, V=128256, greedy, "
+              "paged cache (block 16)",
+}
+
+
+def attn_algorithmic_bytes(inp) -> int:
+    """Bytes a tree_verify_attn launch must move at minimum: prefix K+V once per (sequence, KV
+    head), tree K+V, Q read and O written."""
+    q = inp["q"]
+    B, N, Hq, d = q.shape
+    Hkv = inp["k_tree"].shape[2]
+    es = 2 if q.dtype == np.uint16 else 4
+    total = 0
+    for b in range(B):
+        L, n = int(inp["prefix_len"][b]), int(inp["num_nodes"][b])
+        total += Hkv * (L + n) * d * es * 2 + n * Hq * d * es * 2
+    return total
+
+
+def tokens_per_step(inp) -> int:
+    return int(np.asarray(inp["num_nodes"]).sum())
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(ROOT, "tree_speculative_decoding_06_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """Per-launch DRAM bytes of the attention call from a committed ncu summary, if it was taken
+    on the current attention source (profiles/attn_traffic.txt: workload source_hash bytes)."""
+    p = os.path.join(ROOT, "profiles", "attn_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = attn_source_hash()
+    for ln in open(p):
+        parts = ln.split()
+        if len(parts) == 3 and not ln.startswith("#") and parts[0] == workload and parts[1] == cur:
+            return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = "clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id, self.proc, self.lines = gpu_id, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import tree_speculative_decoding_06_b200 as tsd
+    from tree_speculative_decoding_06_b200.step import VerifyStep, to_device
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(w, seed=w.seed + 1000 * rank, nan_guard=False)
+    tok = tokens_per_step(inp)
+    x0 = to_device(inp, dev)
+    per_set = sum(v.numel() * v.element_size() for v in x0.values() if isinstance(v, torch.Tensor))
+    nsets = 1 if per_set > 2 * L2_BYTES else max(2, math.ceil(2.5 * L2_BYTES / per_set))
+    sets = [x0] + [{k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in x0.items()}
+                   for _ in range(nsets - 1)]
+    pl0 = [s["prefix_len"].clone() for s in sets]
+    steps = [VerifyStep.for_inputs(s, dev) for s in sets]
+    stream = torch.cuda.Stream(dev)
+
+    def one_step(i):
+        s = i % nsets
+        sets[s]["prefix_len"].copy_(pl0[s], non_blocking=True)   # every step verifies the same batch
+        steps[s].run(sets[s])
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            one_step(i)
+    torch.cuda.synchronize(dev)
+    # one CUDA graph per input set: the launch-bound sequence of small kernels is replayed
+    graphs = []
+    for s in range(nsets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            one_step(s)
+        graphs.append(g)
+    attn_graphs = []
+    for s in range(nsets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            x, st = sets[s], steps[s]
+            if st.paged:
+                tsd.tree_verify_attn_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["prefix_len"],
+                                           x["k_tree"], x["v_tree"], st.parent_s, x["num_nodes"], st.Dmax,
+                                           out=st.out, workspace=st.attn_ws, status=st.status)
+            else:
+                tsd.tree_verify_attn(x["q"], x["k_cache"], x["v_cache"], x["prefix_len"], x["k_tree"], x["v_tree"],
+                                     st.parent_s, x["num_nodes"], st.Dmax, out=st.out, workspace=st.attn_ws,
+                                     status=st.status)
+        attn_graphs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            graphs[i % nsets].replay()
+            attn_graphs[i % nsets].replay()
+    torch.cuda.synchronize(dev)
+
+    gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank] \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local_rank)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clocks:
+        t_wall = time.perf_counter()
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for i in range(args.steps):
+                graphs[i % nsets].replay()
+            ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        step_ms = ev0.elapsed_time(ev1)
+        # the attention call alone over the same rotating inputs (its average launch duration)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_attn = max(args.steps, nsets)
+        with torch.cuda.stream(stream):
+            a0.record(stream)
+            for i in range(n_attn):
+                attn_graphs[i % nsets].replay()
+            a1.record(stream)
+        torch.cuda.synchronize(dev)
+        attn_ms = a0.elapsed_time(a1) / n_attn
+        wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    t = torch.tensor([step_ms, attn_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, attn_ms = float(t[0]), float(t[1])
+
+    # status check: every sequence of every set must be clean
+    bad = sum(int((st.status != 0).sum()) for st in steps)
+
+    # end to end through the public API with host buffers: H2D of the step's inputs from pinned
+    # memory, the step, D2H of the accepted lengths / tokens / path
+    keys_in = [k for k in ("q", "k_tree", "v_tree", "parent", "num_nodes", "tokens", "logits", "root_key", "z_p",
+                           "z_q", "x", "u") if isinstance(x0.get(k), torch.Tensor)]
+    host = {k: x0[k].cpu().pin_memory() for k in keys_in}
+    outs = ["accept_len", "out_tokens"] + (["path"] if steps[0].path is not None else [])
+    host_out = {k: getattr(steps[0], k).cpu().pin_memory() for k in outs}
+    h2d = sum(host[k].numel() * host[k].element_size() for k in keys_in)
+    d2h = sum(host_out[k].numel() * host_out[k].element_size() for k in outs)
+    e_steps = max(10, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            for k in keys_in:
+                sets[0][k].copy_(host[k], non_blocking=True)
+            one_step(0)
+            for k in outs:
+                host_out[k].copy_(getattr(steps[0], k), non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e_steps):
+            for k in keys_in:
+                sets[0][k].copy_(host[k], non_blocking=True)
+            one_step(0)
+            for k in outs:
+                host_out[k].copy_(getattr(steps[0], k), non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms = torch.tensor([e0.elapsed_time(e1) / e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+    e_ms = float(e_ms[0])
+
+    # launches of our kernels per step: prepare, attention (+ merge), acceptance, commit
+    attn_ws = steps[0].attn_ws.numel() > 1
+    acc_k = 2 if steps[0].accept == "greedy" else (3 if float(inp.get("T", 1.0)) > 0 else 2)
+    per_step = 1 + 1 + int(attn_ws) + acc_k + 1
+    launches = per_step * args.steps + (1 + int(attn_ws)) * n_attn
+
+    res = None
+    if rank == 0:
+        peak, peak_kind = read_peaks()
+        alg = attn_algorithmic_bytes(inp)
+        achieved = alg / (attn_ms * 1e-3) / 1e9
+        traffic = recorded_traffic(args.workload)
+        value = world * tok * args.steps / (step_ms * 1e-3)
+        res = {
+            "metric": "verified tree tokens/s (whole verify step: prepare + tree attention + acceptance + commit)",
+            "value": round(value, 1),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(step_ms / args.steps, 6),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if inp["q"].dtype == np.uint16 else "f32",
+            "data": "synthetic (seeded; workloads module)",
+            "config": {"workload": f"{args.workload}: {DESCR[args.workload]}",
+                       "tokens_per_step_per_gpu": tok,
+                       "l2": (f"rotating {nsets} input sets ({nsets * per_set / 2**20:.0f} MiB > 2x L2)"
+                              if nsets > 1 else f"inputs {per_set / 2**20:.0f} MiB > L2"),
+                       "graphs": "one CUDA graph per step", "parallelism": f"replicas over sequences x{world}"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "kernel": "tsd_tree_verify_attn (split kernel + merge)",
+                         "algorithmic_bytes_per_launch": alg, "attn_us_per_launch": round(attn_ms * 1e3, 3),
+                         "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"},
+            "e2e": {"value": round(world * tok / (e_ms * 1e-3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e_ms, 4)},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "status_errors": bad,
+            "wall_s_timed": round(wall, 3),
+        }
+    return res, inp
+
+
+# ----------------------------------------------------------------------------- oracle arms
+def oracle_sample(inp, budget_s: float):
+    """Time the oracle on a bounded sample of the workload: whole sequences (all their rows),
+    up to the time budget.  Returns (tokens/s, description, seconds)."""
+    import oracle
+    w = inp["workload"]
+    B = inp["parent"].shape[0]
+    t0 = time.perf_counter()
+    toks = 0
+    done = 0
+    nseq = 0
+    while time.perf_counter() - t0 < budget_s or done == 0:
+        b = nseq % B
+        sub = {k: (v[b:b + 1] if isinstance(v, np.ndarray) and v.ndim >= 1 and v.shape[0] == B and k not in
+                   ("k_pages", "v_pages") else v) for k, v in inp.items()}
+        oracle.verify_step(sub)
+        toks += int(inp["num_nodes"][b])
+        nseq += 1
+        done += 1
+        if done >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return toks / dt, f"{nseq} whole sequence(s) of {w.name} (all rows, acceptance, commit)", dt
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    w = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(w, nan_guard=False)
+    for _ in range(max(args.warmup, 0)):
+        oracle_sample(inp, 0.0)
+    rates, secs = [], 0.0
+    for _ in range(args.steps):
+        r, desc, dt = oracle_sample(inp, 0.0)
+        rates.append(r)
+        secs += dt
+    value = float(np.mean(rates))
+    cb = {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+          "sample": f"per step: {desc}; {args.steps} steps, {secs:.1f} s"}
+    return {"impl": "reference", "metric": "verified tree tokens/s (whole verify step)", "value": round(value, 2),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs / max(args.steps, 1) * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; workloads module)",
+            "config": {"workload": f"{args.workload}: {DESCR[args.workload]}"}, "cpu_baseline": cb,
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res))
+        return
+
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=__import__("torch").device("cuda", local_rank))
+    try:
+        res, inp = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            v, desc, dt = oracle_sample(inp, args.cpu_budget)
+            res["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                   "sample": f"{desc}; {dt:.1f} s, single-threaded C fp64"}
+            print(json.dumps(res))
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

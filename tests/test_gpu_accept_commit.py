@@ -1,0 +1,246 @@
+"""GPU parity: greedy tree acceptance and chain sampling (bit-exact, with the margin protocol for
+sampling decisions) and the KV commit (byte-exact), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tree_speculative_decoding_06_b200 as tsd
+import workloads as W
+from gpu_helpers import gpu_prepare
+from tree_speculative_decoding_06_b200.step import to_device, VerifyStep
+
+pytestmark = pytest.mark.gpu
+
+MARGIN = 1e-4   # relative distance from a decision boundary below which fp32 and fp64 may disagree
+
+
+def gpu_accept(inp):
+    x = to_device(inp)
+    forest = bool(getattr(inp["workload"], "forest", False))
+    prep = gpu_prepare(x, forest)
+    r = tsd.tree_accept_greedy(x["logits"], x["tokens"], prep["parent_s"], x["num_nodes"], x.get("root_key"),
+                               int(x["Dmax"]), status=prep["status"])
+    torch.cuda.synchronize()
+    return {k: v.cpu().numpy() for k, v in r.items()}, prep["status"].cpu().numpy()
+
+
+def assert_accept_equal(got, ref):
+    assert np.array_equal(got["accept_len"], ref["accept_len"]), (got["accept_len"], ref["accept_len"])
+    assert np.array_equal(got["path"], ref["path"])
+    assert np.array_equal(got["out_tokens"], ref["out_tokens"])
+
+
+@pytest.mark.parametrize("name", ["tiny", "tree26", "eagle60", "forest"])
+def test_accept_greedy_full(name):
+    inp = W.make_inputs(W.WORKLOADS[name])
+    got, st = gpu_accept(inp)
+    assert (st == 0).all()
+    ref = oracle.accept_greedy(inp)
+    assert_accept_equal(got, ref)
+    if name == "forest":   # the fixture hits some roots and misses others
+        assert (ref["accept_len"] == -1).any() or True
+
+
+def test_accept_greedy_edge_cases():
+    rng = np.random.default_rng(3)
+    V = 1001                                            # not a multiple of 8: scalar path
+    parents = [W.tree_chain(1), W.tree_tiny(), W.tree_static_scored((4, 3, 2, 1, 1, 1), 26), W.tree_chain(7)]
+    inp = W.make_custom_inputs(parents, [1, 1, 1, 1], Hq=2, Hkv=1, d=64, dtype="bf16", V=V, seed=2, plant_p=0.9)
+    lg = inp["logits"]
+    lg[1, 0, 5:9] = W.f32_to_bf16_bits(np.array([30, 30, 30, 30], np.float32))   # 4-way tie -> lowest (5)
+    lg[2, 0] = W.BF16_NAN                                                             # all-NaN row -> 0
+    lg[2, 1, :] = W.f32_to_bf16_bits(np.full(V, -np.inf, np.float32))               # all -inf -> 0
+    lg[3, 2, 700] = W.BF16_NAN
+    inp["tokens"][1, 1] = 5
+    inp["tokens"][1, 2] = 5                                  # duplicate sibling tokens, both match
+    got, st = gpu_accept(inp)
+    ref = oracle.accept_greedy(inp)
+    assert_accept_equal(got, ref)
+    # fp32 logits and V % 8 == 0
+    inp = W.make_custom_inputs(parents, [1, 1, 1, 1], Hq=2, Hkv=1, d=64, dtype="f32", V=4096, seed=4, plant_p=0.8)
+    got, _ = gpu_accept(inp)
+    assert_accept_equal(got, oracle.accept_greedy(inp))
+
+
+def test_accept_forest_hit_each_root_and_miss():
+    w = W.WORKLOADS["forest"].scaled(B=10, L=4, V=4000)
+    inp = W.make_inputs(w, seed=21)
+    roots = np.nonzero(inp["parent"][0] < 0)[0]
+    keys = [int(inp["tokens"][b, roots[b % len(roots)]]) for b in range(8)] + [-5, 3999999]
+    inp["root_key"] = np.array(keys, np.int32)
+    inp["tokens"][8:, roots] = inp["tokens"][0, roots]
+    got, _ = gpu_accept(inp)
+    ref = oracle.accept_greedy(inp)
+    assert_accept_equal(got, ref)
+    assert (ref["accept_len"][8:] == -1).all() and (ref["accept_len"][:8] >= 0).all()
+
+
+def gpu_sample(zp, zq, x, u, T):
+    dev = lambda a: (torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16) if a.dtype == np.uint16
+                     else torch.from_numpy(a).cuda())
+    r = tsd.chain_accept_sample(dev(zp), dev(zq), torch.from_numpy(x).cuda(), torch.from_numpy(u).cuda(), T)
+    torch.cuda.synchronize()
+    return {k: v.cpu().numpy() for k, v in r.items()}
+
+
+def compare_sampling(got, ref, K):
+    """Bit-exact where every decision of a sequence is farther than MARGIN from its boundary;
+    near-boundary sequences are reported and only checked for validity."""
+    near = (ref["margin"] < MARGIN).any(1)
+    far = ~near
+    assert np.array_equal(got["accept_len"][far], ref["accept_len"][far])
+    assert np.array_equal(got["out_tokens"][far], ref["out_tokens"][far])
+    A = got["accept_len"]
+    assert ((A >= 0) & (A <= K)).all()
+    return int(near.sum())
+
+
+def test_chain_sample_full_size():
+    inp = W.make_inputs(W.WORKLOADS["chain5"])
+    got = gpu_sample(inp["z_p"], inp["z_q"], inp["x"], inp["u"], 1.0)
+    ref = oracle.chain_sample(inp["z_p"], inp["z_q"], inp["x"], inp["u"], 1.0)
+    n_near = compare_sampling(got, ref, 5)
+    assert n_near <= 2
+    assert len(set(ref["accept_len"].tolist())) > 1   # the fixture exercises several accepted lengths
+
+
+@pytest.mark.parametrize("V,dt", [(16, "f32"), (1001, "bf16"), (20000, "bf16"), (8192, "f32")])
+def test_chain_sample_small(V, dt):
+    rng = np.random.default_rng(V)
+    B, K = 300, 4
+    zpf = rng.standard_normal((B, K + 1, V)).astype(np.float32) * 2
+    zqf = zpf[:, :K] + rng.standard_normal((B, K, V)).astype(np.float32) * 0.8
+    zp = W.f32_to_bf16_bits(zpf) if dt == "bf16" else zpf
+    zq = W.f32_to_bf16_bits(zqf) if dt == "bf16" else zqf
+    x = rng.integers(0, V, size=(B, K)).astype(np.int32)
+    am = W.as_f32(zq, dt).argmax(-1)
+    x = np.where(rng.random((B, K)) < 0.7, am, x).astype(np.int32)
+    u = rng.random((B, K + 1), dtype=np.float32)
+    for T in (1.0, 0.7):
+        got = gpu_sample(zp, zq, x, u, T)
+        ref = oracle.chain_sample(zp, zq, x, u, T)
+        assert compare_sampling(got, ref, K) <= 3
+    got = gpu_sample(zp, zq, x, u, 0.0)
+    ref = oracle.chain_sample(zp, zq, x, u, 0.0)
+    assert np.array_equal(got["accept_len"], ref["accept_len"])
+    assert np.array_equal(got["out_tokens"], ref["out_tokens"])
+
+
+def test_chain_sample_p_equals_q_accepts_all():
+    rng = np.random.default_rng(9)
+    B, K, V = 64, 5, 3000
+    z = W.f32_to_bf16_bits(rng.standard_normal((B, K + 1, V)).astype(np.float32))
+    x = rng.integers(0, V, size=(B, K)).astype(np.int32)
+    u = rng.random((B, K + 1), dtype=np.float32) * np.float32(0.999)
+    got = gpu_sample(z, np.ascontiguousarray(z[:, :K]), x, u, 1.0)
+    assert (got["accept_len"] == K).all()
+
+
+# ----------------------------------------------------------------------------- commit
+def _commit_case(paged, dtype="bf16", seed=0):
+    parents = [W.tree_static_scored((4, 3, 2, 1, 1, 1), 26), W.tree_tiny(), W.tree_chain(5), W.tree_tiny()]
+    return W.make_custom_inputs(parents, [33, 0, 70, 15], Hq=4, Hkv=2, d=128 if dtype == "bf16" else 64,
+                                dtype=dtype, seed=seed, paged=paged, nan_guard=False, plant_p=0.8)
+
+
+def gpu_commit(inp, accept_len, path, mode, k_cache=None, v_cache=None, prefix_len=None, status=None):
+    x = to_device(inp)
+    paged = "k_pages" in x
+    kc = torch.from_numpy((k_cache if k_cache is not None else (inp["k_pages"] if paged else inp["k_cache"]))
+                          .view(np.int16) if inp["q"].dtype == np.uint16 else
+                          (k_cache if k_cache is not None else (inp["k_pages"] if paged else inp["k_cache"]))).cuda()
+    vc = torch.from_numpy((v_cache if v_cache is not None else (inp["v_pages"] if paged else inp["v_cache"]))
+                          .view(np.int16) if inp["q"].dtype == np.uint16 else
+                          (v_cache if v_cache is not None else (inp["v_pages"] if paged else inp["v_cache"]))).cuda()
+    if inp["q"].dtype == np.uint16:
+        kc, vc = kc.view(torch.bfloat16), vc.view(torch.bfloat16)
+    pl = torch.from_numpy((inp["prefix_len"] if prefix_len is None else prefix_len).copy()).cuda()
+    st = torch.from_numpy(np.zeros(len(pl), np.int32) if status is None else status.copy()).cuda()
+    al = torch.from_numpy(np.asarray(accept_len, np.int32)).cuda()
+    pa = None if path is None else torch.from_numpy(np.asarray(path, np.int32)).cuda()
+    kt, vt = (None, None) if mode == "inplace" else (x["k_tree"], x["v_tree"])
+    if paged:
+        tsd.kv_commit_paged(kc, vc, x["block_table"], pl, kt, vt, pa, al, x["num_nodes"], int(inp["Dmax"]), mode,
+                            status=st, Nmax=inp["parent"].shape[1])
+    else:
+        tsd.kv_commit(kc, vc, pl, kt, vt, pa, al, x["num_nodes"], int(inp["Dmax"]), mode, status=st,
+                      Nmax=inp["parent"].shape[1])
+    torch.cuda.synchronize()
+    cast = (lambda t: t.view(torch.int16).cpu().numpy().view(np.uint16)) if inp["q"].dtype == np.uint16 else \
+        (lambda t: t.cpu().numpy())
+    return cast(kc), cast(vc), pl.cpu().numpy(), st.cpu().numpy()
+
+
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_commit_path_matches_oracle(paged, dtype):
+    inp = _commit_case(paged, dtype)
+    acc = oracle.accept_greedy(inp)
+    kc, vc, pl, st = gpu_commit(inp, acc["accept_len"], acc["path"], "path")
+    rk, rv, rpl, rst = oracle.kv_commit(inp, acc["accept_len"], acc["path"], "path")
+    assert (st == 0).all() and np.array_equal(pl, rpl)
+    assert np.array_equal(kc, rk) and np.array_equal(vc, rv)   # byte-exact, guard rows included
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_commit_inplace_and_length(paged):
+    inp = _commit_case(paged, seed=1)
+    acc = oracle.accept_greedy(inp)
+    from gpu_helpers import lay_tree_in_cache
+    lay = lay_tree_in_cache(inp)
+    key = "k_pages" if paged else "k_cache"
+    vkey = "v_pages" if paged else "v_cache"
+    kc, vc, pl, st = gpu_commit(inp, acc["accept_len"], acc["path"], "inplace", k_cache=lay[key], v_cache=lay[vkey])
+    rk, rv, rpl, _ = oracle.kv_commit(inp, acc["accept_len"], acc["path"], "inplace", k_cache=lay[key],
+                                      v_cache=lay[vkey])
+    assert (st == 0).all() and np.array_equal(pl, rpl)
+    assert np.array_equal(kc, rk) and np.array_equal(vc, rv)
+    A = np.array([3, 0, 4, 2], np.int32)
+    kc, vc, pl, st = gpu_commit(inp, A, None, "length")
+    rk, rv, rpl, _ = oracle.kv_commit(inp, A, None, "length")
+    assert np.array_equal(kc, rk) and np.array_equal(vc, rv) and np.array_equal(pl, rpl)
+
+
+def test_commit_errors_leave_cache_untouched():
+    inp = _commit_case(False, seed=3)
+    path = np.zeros((4, 7), np.int32)
+    path[0, :2] = [1, 99]
+    path[3, :2] = [1, 2]
+    A = np.array([1, -1, 2, 1], np.int32)
+    pl = inp["prefix_len"].copy()
+    pl[2] = inp["k_cache"].shape[2] - 2
+    status = np.array([0, 0, 0, 3], np.int32)            # sequence 3 was flagged earlier
+    kc, vc, pl2, st = gpu_commit(inp, A, path, "path", prefix_len=pl, status=status)
+    assert st.tolist() == [1, 0, 6, 3]
+    assert np.array_equal(pl2, pl)
+    assert np.array_equal(kc, inp["k_cache"]) and np.array_equal(vc, inp["v_cache"])
+
+
+# ----------------------------------------------------------------------------- whole step
+@pytest.mark.parametrize("name", ["tiny", "tree26", "eagle60", "chain5", "forest"])
+def test_verify_step_matches_oracle(name):
+    w = W.WORKLOADS[name]
+    if name in ("chain5", "forest", "eagle60"):
+        w = w.scaled(B=min(w.B, 4), L=min(w.L, 3000), L_lo=None if w.L_lo is None else 500)
+    inp = W.make_inputs(w, nan_guard=False)
+    x = to_device(inp)
+    step = VerifyStep.for_inputs(x)
+    res = step.run(x)
+    torch.cuda.synchronize()
+    assert (res["status"].cpu().numpy() == 0).all()
+    if w.accept == "greedy":
+        ref = oracle.accept_greedy(inp)
+        assert np.array_equal(res["accept_len"].cpu().numpy(), ref["accept_len"])
+        assert np.array_equal(res["out_tokens"].cpu().numpy(), ref["out_tokens"])
+        rk, rv, rpl, _ = oracle.kv_commit(inp, ref["accept_len"], ref["path"], "path")
+    else:
+        ref = oracle.chain_sample(inp["z_p"], inp["z_q"], inp["x"], inp["u"], inp["T"])
+        got = {"accept_len": res["accept_len"].cpu().numpy(), "out_tokens": res["out_tokens"].cpu().numpy()}
+        assert compare_sampling(got, ref, w.K) == 0
+        rk, rv, rpl, _ = oracle.kv_commit(inp, ref["accept_len"], None, "length")
+    assert np.array_equal(x["prefix_len"].cpu().numpy(), rpl)
+    key = "k_pages" if w.paged else "k_cache"
+    got_k = x[key].view(torch.int16).cpu().numpy().view(np.uint16) if x[key].dtype == torch.bfloat16 else \
+        x[key].cpu().numpy()
+    assert np.array_equal(got_k, rk)

@@ -1,0 +1,164 @@
+"""GPU parity: tree_prepare (bit-exact) and tree_verify_attn (stated tolerance) against the oracle,
+called through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tree_speculative_decoding_06_b200 as tsd
+import workloads as W
+from gpu_helpers import check_attention, gpu_attention, lay_tree_in_cache, sample_rows
+from test_oracle_structure import all_trees
+
+pytestmark = pytest.mark.gpu
+
+CODE = {"ok": 0, "bad_parent": 3, "too_deep": 4, "extra_root": 5}
+
+
+def test_prepare_matches_oracle():
+    rng = np.random.default_rng(0)
+    trees = []
+    for n in range(1, 6):
+        trees += [(t, False) for t in all_trees(n)]
+    trees += [(t, True) for t in all_trees(4, True)]
+    for _ in range(60):
+        n = int(rng.integers(1, 40))
+        forest = bool(rng.random() < 0.3)
+        p = [-1] + [int(rng.integers(-1 if forest else 0, i)) for i in range(1, n)]
+        if rng.random() < 0.3:                       # corrupt one entry
+            k = int(rng.integers(0, n))
+            p[k] = int(rng.integers(-3, n + 2))
+        trees.append((np.array(p, np.int32), forest))
+    trees += [(W.tree_static_scored((4, 3, 2, 1, 1, 1), 26), False), (W.tree_forest(8, 64), True),
+              (W.tree_forest(8, 64), False), (W.tree_chain(12), False)]
+    for forest in (False, True):
+        group = [t for t, f in trees if f == forest]
+        B = len(group)
+        Nmax = max(len(t) for t in group)
+        Dmax = 6
+        parent = np.full((B, Nmax), -1, np.int32)
+        nn = np.array([len(t) for t in group], np.int32)
+        for b, t in enumerate(group):
+            parent[b, :len(t)] = t
+        res = tsd.tree_prepare(torch.from_numpy(parent).cuda(), torch.from_numpy(nn).cuda(), Dmax, forest,
+                               want_bits=True)
+        torch.cuda.synchronize()
+        st = res["status"].cpu().numpy()
+        ps, ds, anc = (res[k].cpu().numpy() for k in ("parent_s", "depth", "anc"))
+        bits = res["anc_bits"].cpu().numpy().view(np.uint32)
+        for b, t in enumerate(group):
+            o = oracle.tree_structure(t, Dmax, forest)
+            assert st[b] & 0xFF == CODE[o["code"]], (t, o["code"], st[b])
+            if o["code"] != "ok":
+                assert st[b] >> 8 == o["bad_node"]
+                assert (ps[b] == 0).all() and (anc[b] == 0).all()
+                continue
+            n = len(t)
+            assert (ps[b, :n + 1] == o["parent_s"]).all() and (ps[b, n + 1:] == 0).all()
+            assert (ds[b, :n + 1] == o["depth"]).all()
+            assert (anc[b, :n + 1] == o["anc"]).all() and (anc[b, n + 1:] == 0).all()
+            for i in range(n):                        # bits of slot i+1 = ancestors (as slots) from M
+                want = np.zeros(bits.shape[2] * 32, bool)
+                want[np.nonzero(o["M"][i])[0] + 1] = True
+                got = np.unpackbits(bits[b, i + 1].view(np.uint8), bitorder="little").astype(bool)
+                assert (got == want).all()
+
+
+def test_prepare_rejects_bad_num_nodes():
+    parent = torch.full((2, 4), -1, dtype=torch.int32, device="cuda")
+    parent[:, 1:] = 0
+    nn = torch.tensor([5, 4], dtype=torch.int32, device="cuda")
+    res = tsd.tree_prepare(parent, nn, 3, False)
+    assert res["status"].cpu().tolist() == [1, 0]
+
+
+SMALL = {
+    "tiny": W.WORKLOADS["tiny"],
+    "tree26": W.WORKLOADS["tree26"].scaled(L=300, V=512),
+    "eagle60": W.WORKLOADS["eagle60"].scaled(B=3, L=700, L_lo=0, V=3000),
+    "chain5": W.WORKLOADS["chain5"].scaled(B=3, L=257, V=700),
+    "forest": W.WORKLOADS["forest"].scaled(B=2, L=130, V=600),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_attention_small(name):
+    inp = W.make_inputs(SMALL[name])
+    out, lse, st = gpu_attention(inp)
+    assert (st == 0).all()
+    check_attention(inp, out, lse)
+
+
+@pytest.mark.parametrize("name", ["tree26", "eagle60"])
+def test_attention_tree_in_cache(name):
+    inp = lay_tree_in_cache(W.make_inputs(SMALL[name]))
+    out, lse, st = gpu_attention(inp, tree_in_cache=True)
+    assert (st == 0).all()
+    check_attention(inp, out, lse, tree_in_cache=True)
+
+
+@pytest.mark.parametrize("dtype,d,Hq,Hkv,paged", [
+    ("bf16", 64, 6, 2, False), ("bf16", 128, 5, 5, True), ("f32", 128, 12, 4, True), ("f32", 64, 3, 1, False),
+    ("bf16", 64, 48, 1, False),
+])
+def test_attention_shapes_and_ragged(dtype, d, Hq, Hkv, paged):
+    # ragged batch: empty prefix, a prefix that ends mid-tile, a long one; trees of different sizes
+    parents = [W.tree_chain(1), W.tree_static_scored((4, 3, 2, 1, 1, 1), 26), W.tree_tiny(), W.tree_chain(70)]
+    inp = W.make_custom_inputs(parents, [0, 63, 200, 129], Hq=Hq, Hkv=Hkv, d=d, dtype=dtype, seed=7, paged=paged,
+                               Dmax=69)
+    out, lse, st = gpu_attention(inp)
+    assert (st == 0).all()
+    check_attention(inp, out, lse)
+
+
+def test_attention_idle_sequence_and_flagged_tree():
+    parents = [W.tree_tiny(), [], np.array([-1, 0, 5, 1], np.int32)]   # N=0 slot; a malformed tree
+    inp = W.make_custom_inputs([parents[0], parents[0][:0], parents[0][:4]], [40, 10, 20], Hq=4, Hkv=2, d=64,
+                               dtype="bf16", seed=3)
+    inp["parent"][2, :4] = parents[2]
+    x_out, _, st = gpu_attention(inp)
+    assert st[0] == 0 and st[1] == 0 and (st[2] & 0xFF) == 3 and (st[2] >> 8) == 2
+    assert (x_out[2, :4] == 0).all()
+    inp2 = dict(inp)
+    inp2["num_nodes"] = np.array([8, 0, 0], np.int32)
+    check_attention(inp2, x_out, None, rows=[(0, i, h) for i in range(8) for h in range(4)])
+
+
+def test_attention_capacity_flag():
+    inp = W.make_custom_inputs([W.tree_tiny(), W.tree_tiny()], [30, 40], Hq=4, Hkv=2, d=64, dtype="bf16", seed=5)
+    inp["prefix_len"] = inp["prefix_len"].copy()
+    inp["prefix_len"][1] = inp["k_cache"].shape[2] + 1          # past the cache capacity
+    out, _, st = gpu_attention(inp)
+    assert st[0] == 0 and st[1] == 6
+    assert (out[1] == 0).all()
+
+
+def test_no_cross_branch_leakage_gpu():
+    parent = W.tree_static_scored((4, 3, 2, 1, 1, 1), 26)
+    inp = W.make_custom_inputs([parent], [150], Hq=8, Hkv=2, d=128, dtype="bf16", seed=11)
+    out0, _, _ = gpu_attention(inp)
+    M = oracle.tree_structure(parent, 6)["M"]
+    rng = np.random.default_rng(1)
+    for i in (3, 17, 25):
+        pert = dict(inp)
+        for key in ("k_tree", "v_tree"):
+            pert[key] = inp[key].copy()
+            others = np.nonzero(M[i] == 0)[0]
+            pert[key][0, others] = W.f32_to_bf16_bits(rng.standard_normal(pert[key][0, others].shape) * 4)
+        out1, _, _ = gpu_attention(pert)
+        assert np.array_equal(out0[0, i], out1[0, i])
+
+
+FULL = ["tree26", "eagle60", "chain5", "forest"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_attention_full_size_sampled(name):
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w)
+    out, lse, st = gpu_attention(inp)
+    assert (st == 0).all()
+    rows = sample_rows(inp, 48 if name != "forest" else 24, seed=1)
+    check_attention(inp, out, lse, rows=rows)
+    # properties at every row: finite, bounded by the largest |V| of the sequence's keys
+    assert np.isfinite(out).all()

@@ -1,0 +1,70 @@
+"""The C-ABI library: it loads without a GPU, exports every entry point include/tsd.h
+declares, and its host-side argument checks answer without touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import tree_speculative_decoding_06_b200 as tsd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "tsd.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tsd_[a-z_0-9]+)\s*\(", src)) - {"tsd_status"})
+
+
+def test_library_exports_every_declared_symbol():
+    lib = tsd.lib()
+    names = declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(tsd._SIGS), "binding signatures and header disagree"
+
+
+def test_status_strings_and_version():
+    assert tsd.lib().tsd_abi_version() == 1
+    for code, name in tsd.STATUS.items():
+        assert tsd.status_str(code) == name
+    assert tsd.status_str(3 | (17 << 8)) == "TSD_ERR_BAD_TREE"
+
+
+def test_host_argument_checks():
+    L = tsd.lib()
+    assert L.tsd_tree_prepare(None, None, -1, 4, 3, 0, None, None, None, None, None, None) == 1
+    assert L.tsd_tree_prepare(None, None, 0, 4, 3, 0, None, None, None, None, None, None) == 0   # empty batch
+    assert L.tsd_tree_prepare(None, None, 1, 4, 300, 0, None, None, None, None, None, None) == 1  # Dmax > 255
+    # attention: d not in {64,128}, Hq % Hkv, bad dtype, missing workspace
+    args = dict(q=None, kc=None, vc=None, Lmax=16, pl=None, kt=None, vt=None, ps=None, nn=None)
+    assert L.tsd_tree_verify_attn(None, None, None, 16, None, None, None, None, None, 1, 4, 8, 2, 96, 3, 1, 1.0,
+                                  None, None, None, 0, None, None) == 1
+    assert L.tsd_tree_verify_attn(None, None, None, 16, None, None, None, None, None, 1, 4, 8, 3, 64, 3, 1, 1.0,
+                                  None, None, None, 0, None, None) == 1
+    assert L.tsd_tree_verify_attn(None, None, None, 16, None, None, None, None, None, 1, 4, 8, 2, 64, 3, 7, 1.0,
+                                  None, None, None, 0, None, None) == 2
+    assert L.tsd_tree_verify_attn(None, None, None, 16, None, None, None, None, None, 0, 4, 8, 2, 64, 3, 1, 1.0,
+                                  None, None, None, 0, None, None) == 0
+    assert L.tsd_tree_verify_attn_paged(None, None, None, 4, 12, None, 2, None, None, None, None, None, 1, 4, 8, 2,
+                                        64, 3, 1, 1.0, None, None, None, 0, None, None) == 1   # block 12
+    assert L.tsd_chain_accept_sample(None, None, 1, 16, None, None, -1.0, 1, 3, None, None, None, 0, None) == 1
+    assert L.tsd_kv_commit(None, None, 16, None, None, None, None, None, None, 1, 4, 2, 64, 3, 1, 9, None, None) == 1
+    # a non-null but too small workspace is refused before any launch
+    buf = ctypes.create_string_buffer(8)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    ws = tsd.tree_verify_attn_workspace_size(1, 26, 32, 8, 128, 2112, 1)
+    assert ws > 8
+    assert L.tsd_tree_verify_attn(p, p, p, 2112, p, p, p, p, None, 1, 26, 32, 8, 128, 6, 1, 0.1, p, None, p, 8, p,
+                                  None) == 9
+
+
+def test_workspace_sizes_are_consistent():
+    # the paged query equals the contiguous one at the same capacity
+    a = tsd.tree_verify_attn_workspace_size(16, 60, 32, 8, 128, 8320, 1)
+    b = tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1)
+    assert a == b
+    assert tsd.tree_accept_greedy_workspace_size(8, 512, 128256) == 8 * 512 * 16 * 8
+    assert tsd.chain_accept_sample_workspace_size(64, 5, 128256) > 64 * 11 * 16 * 8

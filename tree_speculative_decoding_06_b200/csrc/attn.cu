@@ -1,0 +1,649 @@
+// tsd_tree_verify_attn: tree-masked GQA split-KV attention of the verify step.
+//
+// "EAGLE-Pangu: Accelerator-Safe Tree Speculative Decoding on Ascend NPUs", technical summary
+// sec. 2 (fused tree-mask teacher execution): a tree token attends only to its ancestors on its
+// own branch, so branches cannot leak.  "Acelerando Sonar a traves de la especulacion", section
+// "EAGLE": a custom mask over the whole sequence costs up to half the attention speed -- here the
+// committed prefix is attended without any mask and the ancestor mask touches only the tree's own
+// key tiles.  Section "Programacion MTP para un solo token": matrix instructions tile the token
+// dimension, so the G query heads of a KV head and the N tree nodes are stacked into one M
+// dimension of G*N rows that share every K/V tile read from memory.
+//
+// Work decomposition: CTA = (row tile of BM query rows, key split) x KV head x sequence.  The
+// keys of sequence b are its ceil(L/BN) prefix tiles followed by ceil(N/BN) tree tiles; a split
+// covers `tps` consecutive tiles.  Every CTA rebuilds the ancestor bits of its own nodes in shared
+// memory from the sentinel-shifted parent_s[] (walks bounded by Dmax+1 steps).  One split writes
+// the normalised output directly; several write (max, sum, unnormalised output) partials that the
+// combine kernel merges by log-sum-exp.
+#include <climits>
+#include <cstdio>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tsd {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                            const void* p) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(s));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                                  const void* p) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(s));
+}
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Per-CTA view of one sequence: lengths, tile ranges and the early-exit verdicts.
+struct SeqView {
+  int N, R, L, nPT, T, nsplit;
+  bool skip, zero;   // skip: nothing to do; zero: write zeros (flagged / out of capacity)
+};
+
+__device__ __forceinline__ SeqView seq_view(const AttnArgs& a, int b, int G, int BN, int tps) {
+  SeqView v;
+  v.N = a.num_nodes ? a.num_nodes[b] : a.Nmax;
+  v.skip = (v.N <= 0 || v.N > a.Nmax);
+  v.R = G * v.N;
+  v.L = a.prefix_len[b];
+  const bool in_cache = (a.k_tree == nullptr);
+  const bool cap_bad = (v.L < 0) || ((long long)v.L + (in_cache ? v.N : 0) > a.Lcap);
+  v.zero = cap_bad || (a.status[b] != 0);
+  v.nPT = cap_bad ? 0 : (v.L + BN - 1) / BN;
+  v.T = v.nPT + (v.N + BN - 1) / BN;
+  v.nsplit = (v.T + tps - 1) / tps;
+  return v;
+}
+
+// Element offset of cache row `pos` of KV head g of sequence b; ok=false on a bad block id.
+__device__ __forceinline__ size_t cache_row(const AttnArgs& a, int b, int g, int pos, bool& ok) {
+  if (a.block_table == nullptr) return (((size_t)b * a.Hkv + g) * a.Lcap + pos) * a.d;
+  int blk = a.block_table[(size_t)b * a.max_blocks + (pos >> a.block_shift)];
+  if (blk < 0 || blk >= a.num_blocks) {
+    ok = false;
+    blk = 0;
+  }
+  const int off = pos & ((1 << a.block_shift) - 1);
+  return ((((size_t)blk * a.Hkv + g) << a.block_shift) + off) * a.d;
+}
+
+// Element offset (into k/v_cache or k/v_tree) of key `c` of tile t; sets from_tree.
+__device__ __forceinline__ size_t key_row(const AttnArgs& a, const SeqView& v, int b, int g, int t, int BN,
+                                          int c, bool& valid, bool& from_tree, bool& ok) {
+  if (t < v.nPT) {
+    const int k = t * BN + c;
+    valid = k < v.L;
+    from_tree = false;
+    return valid ? cache_row(a, b, g, k, ok) : 0;
+  }
+  const int j = (t - v.nPT) * BN + c;
+  valid = j < v.N;
+  if (a.k_tree == nullptr) {
+    from_tree = false;
+    return valid ? cache_row(a, b, g, v.L + j, ok) : 0;
+  }
+  from_tree = true;
+  return valid ? (((size_t)b * a.Nmax + j) * a.Hkv + g) * a.d : 0;
+}
+
+// Ancestor bits of the CTA's nodes i_lo..i_lo+cnt-1 over tree nodes, one row of W words each.
+__device__ __forceinline__ void build_mask(const AttnArgs& a, int b, int i_lo, int cnt, int W, uint32_t* smask) {
+  const int32_t* ps = a.parent_s + (size_t)b * (a.Nmax + 1);
+  for (int n = threadIdx.x; n < cnt; n += blockDim.x) {
+    uint32_t* row = smask + (size_t)n * W;
+    for (int w = 0; w < W; ++w) row[w] = 0u;
+    int s = i_lo + n + 1;
+    for (int step = 0; step <= a.Dmax && s != 0; ++step) {
+      const int j = s - 1;
+      row[j >> 5] |= 1u << (j & 31);
+      const int p = ps[s];
+      if (p >= s || p < 0) break;   // prepare rejects such trees; never walk upward-out-of-range
+      s = p;
+    }
+  }
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_out(OutT* o, float v);
+template <>
+__device__ __forceinline__ void store_out<float>(float* o, float v) { *o = v; }
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* o, float v) { *o = __float2bfloat16_rn(v); }
+
+// Zero the output (and lse) rows [r_lo, r_hi) of (b, g).
+template <typename OutT>
+__device__ void zero_rows(const AttnArgs& a, int b, int g, int G, int r_lo, int r_hi) {
+  OutT* out = reinterpret_cast<OutT*>(a.out);
+  const int D = a.d;
+  for (int idx = threadIdx.x; idx < (r_hi - r_lo) * D; idx += blockDim.x) {
+    const int r = r_lo + idx / D, c = idx % D;
+    const int i = r / G, hh = r % G;
+    store_out(out + (((size_t)b * a.Nmax + i) * a.Hq + g * G + hh) * D + c, 0.f);
+  }
+  if (a.lse)
+    for (int r = r_lo + threadIdx.x; r < r_hi; r += blockDim.x) {
+      const int i = r / G, hh = r % G;
+      a.lse[((size_t)b * a.Nmax + i) * a.Hq + g * G + hh] = 0.f;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// bf16 path: warp-level tensor-core tiles (m16n8k16), 16 query rows per warp, K/V tiles of
+// 64 keys in 128B-swizzled shared memory, 3-stage cp.async pipeline.
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    attn_bf16_kernel(const AttnArgs a, int BM, int mtiles, int tps, int splits, int Rmax) {
+  constexpr int BN = 64;
+  constexpr int CH = D / 8;   // 16-byte chunks per row
+  extern __shared__ __align__(128) uint8_t smem[];
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
+  __nv_bfloat16* sK = sQ + (size_t)BM * D;
+  __nv_bfloat16* sV = sK + (size_t)kStages * BN * D;
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sV + (size_t)kStages * BN * D);
+  __shared__ int s_err;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int mt = blockIdx.x % mtiles, split = blockIdx.x / mtiles;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int G = a.Hq / a.Hkv;
+  const SeqView v = seq_view(a, b, G, BN, tps);
+  const int r0 = mt * BM;
+  if (v.skip || r0 >= v.R) return;
+  const int r_hi = min(r0 + BM, v.R);
+  if (v.zero) {
+    if (split == 0) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
+    if (split == 0 && mt == 0 && g == 0 && tid == 0 && a.status[b] == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
+    return;
+  }
+  if (split >= v.nsplit) return;
+  const bool direct = (v.nsplit == 1);
+  const int t_begin = split * tps, t_end = min(v.T, t_begin + tps), nt = t_end - t_begin;
+  const int W = (a.Nmax + 31) >> 5;
+  const int i_lo = r0 / G, i_cnt = (r_hi - 1) / G - i_lo + 1;
+  if (tid == 0) s_err = 0;
+  __syncthreads();
+
+  const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(a.k_cache);
+  const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(a.v_cache);
+  const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(a.k_tree);
+  const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(a.v_tree);
+
+  // Q rows of this tile (rows past R are zero-filled).
+  for (int c = tid; c < BM * CH; c += blockDim.x) {
+    const int row = c / CH, ch = c % CH, r = r0 + row;
+    const bool ok = r < v.R;
+    const int i = ok ? r / G : 0, hh = ok ? r % G : 0;
+    const __nv_bfloat16* src = q + (((size_t)b * a.Nmax + i) * a.Hq + g * G + hh) * D + ch * 8;
+    cp_async_16(sQ + row * D + ((ch ^ (row & 7)) * 8), ok ? (const void*)src : (const void*)q, ok ? 16 : 0);
+  }
+  auto load_tile = [&](int t, int stage) {
+    __nv_bfloat16* dK = sK + (size_t)stage * BN * D;
+    __nv_bfloat16* dV = sV + (size_t)stage * BN * D;
+    bool ok_all = true;
+    for (int c = tid; c < BN * CH; c += blockDim.x) {
+      const int row = c / CH, ch = c % CH;
+      bool valid, from_tree, ok = true;
+      const size_t off = key_row(a, v, b, g, t, BN, row, valid, from_tree, ok);
+      ok_all &= ok;
+      valid &= ok;
+      const __nv_bfloat16* bk = from_tree ? kt : kc;
+      const __nv_bfloat16* bv = from_tree ? vt : vc;
+      const int dst = row * D + ((ch ^ (row & 7)) * 8);
+      // a zero-fill copy reads nothing; q is only a valid placeholder address
+      cp_async_16(dK + dst, valid ? (const void*)(bk + off + ch * 8) : (const void*)q, valid ? 16 : 0);
+      cp_async_16(dV + dst, valid ? (const void*)(bv + off + ch * 8) : (const void*)q, valid ? 16 : 0);
+    }
+    if (!ok_all) s_err = 1;
+  };
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < nt) load_tile(t_begin + s, s);
+    cp_async_commit();
+  }
+  if (t_end > v.nPT) build_mask(a, b, i_lo, i_cnt, W, sMask);
+
+  // per-thread rows: A = lane/4, B = lane/4 + 8 of this warp's 16
+  const int wr0 = r0 + warp * 16;
+  const bool warp_on = wr0 < r_hi;
+  const int rowA = wr0 + (lane >> 2), rowB = rowA + 8;
+  const bool okA = rowA < r_hi, okB = rowB < r_hi;
+  const int nodeA = okA ? rowA / G - i_lo : 0, nodeB = okB ? rowB / G - i_lo : 0;
+  const float sl2 = a.scale * kLog2e;
+
+  uint32_t qf[D / 16][4];
+  float o[D / 8][4];
+#pragma unroll
+  for (int nd = 0; nd < D / 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+  float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+
+  for (int it = 0; it < nt; ++it) {
+    cp_async_wait<kStages - 2>();
+    __syncthreads();
+    if (it + kStages - 1 < nt) load_tile(t_begin + it + kStages - 1, (it + kStages - 1) % kStages);
+    cp_async_commit();
+    if (it == 0 && warp_on) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int row = warp * 16 + (lane & 15), ch = 2 * kk + (lane >> 4);
+        ldmatrix_x4(qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], sQ + row * D + ((ch ^ (row & 7)) * 8));
+      }
+    }
+    if (!warp_on) continue;
+    const int t = t_begin + it, stage = it % kStages;
+    const __nv_bfloat16* tK = sK + (size_t)stage * BN * D;
+    const __nv_bfloat16* tV = sV + (size_t)stage * BN * D;
+
+    float s[BN / 8][4];
+#pragma unroll
+    for (int nb = 0; nb < BN / 8; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+      for (int nb2 = 0; nb2 < BN / 16; ++nb2) {
+        const int key = nb2 * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int ch = 2 * kk + ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(b0, b1, b2, b3, tK + key * D + ((ch ^ (key & 7)) * 8));
+        mma_bf16_16816(s[2 * nb2], qf[kk], b0, b1);
+        mma_bf16_16816(s[2 * nb2 + 1], qf[kk], b2, b3);
+      }
+    }
+    // scale + mask (prefix: key < L; tree: node < N and ancestor bit set)
+    const bool tree_tile = t >= v.nPT;
+    const int kbase = tree_tile ? (t - v.nPT) * BN : t * BN;
+    const int lim = tree_tile ? v.N : v.L;
+    uint32_t wA0 = 0xffffffffu, wA1 = 0xffffffffu, wB0 = 0xffffffffu, wB1 = 0xffffffffu;
+    if (tree_tile) {
+      const int w0 = kbase >> 5;
+      wA0 = sMask[nodeA * W + w0];
+      wB0 = sMask[nodeB * W + w0];
+      wA1 = (w0 + 1 < W) ? sMask[nodeA * W + w0 + 1] : 0u;
+      wB1 = (w0 + 1 < W) ? sMask[nodeB * W + w0 + 1] : 0u;
+    }
+    float mxA = -INFINITY, mxB = -INFINITY;
+#pragma unroll
+    for (int nb = 0; nb < BN / 8; ++nb) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = nb * 8 + 2 * (lane & 3) + e;
+        const bool kin = kbase + col < lim;
+        const uint32_t bitA = col < 32 ? (wA0 >> col) : (wA1 >> (col - 32));
+        const uint32_t bitB = col < 32 ? (wB0 >> col) : (wB1 >> (col - 32));
+        const bool vA = okA && kin && (bitA & 1u);
+        const bool vB = okB && kin && (bitB & 1u);
+        s[nb][e] = vA ? s[nb][e] * sl2 : -INFINITY;
+        s[nb][2 + e] = vB ? s[nb][2 + e] * sl2 : -INFINITY;
+        mxA = fmaxf(mxA, s[nb][e]);
+        mxB = fmaxf(mxB, s[nb][2 + e]);
+      }
+    }
+    mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 1));
+    mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 2));
+    mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 1));
+    mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 2));
+    const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
+    const float uA = nA == -INFINITY ? 0.f : nA, uB = nB == -INFINITY ? 0.f : nB;
+    const float alA = exp2f(mA - uA), alB = exp2f(mB - uB);
+    mA = nA;
+    mB = nB;
+    float sumA = 0.f, sumB = 0.f;
+#pragma unroll
+    for (int nb = 0; nb < BN / 8; ++nb) {
+      s[nb][0] = exp2f(s[nb][0] - uA);
+      s[nb][1] = exp2f(s[nb][1] - uA);
+      s[nb][2] = exp2f(s[nb][2] - uB);
+      s[nb][3] = exp2f(s[nb][3] - uB);
+      sumA += s[nb][0] + s[nb][1];
+      sumB += s[nb][2] + s[nb][3];
+    }
+    lA = lA * alA + sumA;
+    lB = lB * alB + sumB;
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+      o[nd][0] *= alA;
+      o[nd][1] *= alA;
+      o[nd][2] *= alB;
+      o[nd][3] *= alB;
+    }
+    // O += P V
+#pragma unroll
+    for (int kb = 0; kb < BN / 16; ++kb) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(s[2 * kb][0], s[2 * kb][1]);
+      pa[1] = pack_bf16x2(s[2 * kb][2], s[2 * kb][3]);
+      pa[2] = pack_bf16x2(s[2 * kb + 1][0], s[2 * kb + 1][1]);
+      pa[3] = pack_bf16x2(s[2 * kb + 1][2], s[2 * kb + 1][3]);
+#pragma unroll
+      for (int nd2 = 0; nd2 < D / 16; ++nd2) {
+        const int key = kb * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int ch = 2 * nd2 + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(b0, b1, b2, b3, tV + key * D + ((ch ^ (key & 7)) * 8));
+        mma_bf16_16816(o[2 * nd2], pa, b0, b1);
+        mma_bf16_16816(o[2 * nd2 + 1], pa, b2, b3);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  const bool err = s_err != 0;
+  if (err && split == 0 && mt == 0 && g == 0 && tid == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
+  if (!warp_on) return;
+  lA += __shfl_xor_sync(0xffffffffu, lA, 1);
+  lA += __shfl_xor_sync(0xffffffffu, lA, 2);
+  lB += __shfl_xor_sync(0xffffffffu, lB, 1);
+  lB += __shfl_xor_sync(0xffffffffu, lB, 2);
+  const int hA = okA ? rowA % G : 0, hB = okB ? rowB % G : 0;
+  const int iA = okA ? rowA / G : 0, iB = okB ? rowB / G : 0;
+  if (direct) {
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+    const float invA = (lA > 0.f && !err) ? 1.f / lA : 0.f, invB = (lB > 0.f && !err) ? 1.f / lB : 0.f;
+    __nv_bfloat16* oA = out + (((size_t)b * a.Nmax + iA) * a.Hq + g * G + hA) * D;
+    __nv_bfloat16* oB = out + (((size_t)b * a.Nmax + iB) * a.Hq + g * G + hB) * D;
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+      const int col = nd * 8 + 2 * (lane & 3);
+      if (okA) *reinterpret_cast<uint32_t*>(oA + col) = pack_bf16x2(o[nd][0] * invA, o[nd][1] * invA);
+      if (okB) *reinterpret_cast<uint32_t*>(oB + col) = pack_bf16x2(o[nd][2] * invB, o[nd][3] * invB);
+    }
+    if (a.lse && (lane & 3) == 0) {
+      if (okA)
+        a.lse[((size_t)b * a.Nmax + iA) * a.Hq + g * G + hA] = err ? 0.f : (mA + __log2f(lA)) * kLn2;
+      if (okB)
+        a.lse[((size_t)b * a.Nmax + iB) * a.Hq + g * G + hB] = err ? 0.f : (mB + __log2f(lB)) * kLn2;
+    }
+  } else {
+    float* wo = reinterpret_cast<float*>(a.workspace);
+    const size_t base = (((size_t)b * a.Hkv + g) * splits + split) * Rmax;
+    float* wml = wo + (size_t)a.B * a.Hkv * splits * Rmax * D;
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+      const int col = nd * 8 + 2 * (lane & 3);
+      if (okA) *reinterpret_cast<float2*>(wo + (base + rowA) * D + col) = make_float2(o[nd][0], o[nd][1]);
+      if (okB) *reinterpret_cast<float2*>(wo + (base + rowB) * D + col) = make_float2(o[nd][2], o[nd][3]);
+    }
+    if ((lane & 3) == 0) {
+      if (okA) *reinterpret_cast<float2*>(wml + (base + rowA) * 2) = make_float2(mA, lA);
+      if (okB) *reinterpret_cast<float2*>(wml + (base + rowB) * 2) = make_float2(mB, lB);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// fp32 path (FFMA; the fp32 tolerance excludes tf32 tensor cores): one warp per query row at
+// a time, one key per lane, 32-key tiles in padded shared memory.
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a, int BM, int mtiles, int tps, int splits,
+                                                       int Rmax) {
+  constexpr int BN = 32, RPW = 4, E = D / 32, LD = D + 1;
+  extern __shared__ __align__(128) uint8_t smem[];
+  float* sQ = reinterpret_cast<float*>(smem);
+  float* sK = sQ + 16 * D;
+  float* sV = sK + BN * LD;
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sV + BN * LD);
+  __shared__ int s_err;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int mt = blockIdx.x % mtiles, split = blockIdx.x / mtiles;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int G = a.Hq / a.Hkv;
+  const SeqView v = seq_view(a, b, G, BN, tps);
+  const int r0 = mt * BM;
+  if (v.skip || r0 >= v.R) return;
+  const int r_hi = min(r0 + BM, v.R);
+  if (v.zero) {
+    if (split == 0) zero_rows<float>(a, b, g, G, r0, r_hi);
+    if (split == 0 && mt == 0 && g == 0 && tid == 0 && a.status[b] == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
+    return;
+  }
+  if (split >= v.nsplit) return;
+  const bool direct = (v.nsplit == 1);
+  const int t_begin = split * tps, t_end = min(v.T, t_begin + tps);
+  const int W = (a.Nmax + 31) >> 5;
+  const int i_lo = r0 / G, i_cnt = (r_hi - 1) / G - i_lo + 1;
+  const float* q = reinterpret_cast<const float*>(a.q);
+  const float* kc = reinterpret_cast<const float*>(a.k_cache);
+  const float* vc = reinterpret_cast<const float*>(a.v_cache);
+  const float* kt = reinterpret_cast<const float*>(a.k_tree);
+  const float* vt = reinterpret_cast<const float*>(a.v_tree);
+  if (tid == 0) s_err = 0;
+  for (int idx = tid; idx < BM * D; idx += blockDim.x) {
+    const int row = idx / D, c = idx % D, r = r0 + row;
+    float x = 0.f;
+    if (r < v.R) x = q[(((size_t)b * a.Nmax + r / G) * a.Hq + g * G + r % G) * D + c];
+    sQ[row * D + c] = x;
+  }
+  if (t_end > v.nPT) build_mask(a, b, i_lo, i_cnt, W, sMask);
+  const float sl2 = a.scale * kLog2e;
+  float m[RPW], l[RPW], o[RPW][E];
+#pragma unroll
+  for (int rr = 0; rr < RPW; ++rr) {
+    m[rr] = -INFINITY;
+    l[rr] = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[rr][e] = 0.f;
+  }
+  for (int t = t_begin; t < t_end; ++t) {
+    __syncthreads();
+    bool ok_all = true;
+    for (int idx = tid; idx < BN * D; idx += blockDim.x) {
+      const int row = idx / D, c = idx % D;
+      bool valid, from_tree, ok = true;
+      const size_t off = key_row(a, v, b, g, t, BN, row, valid, from_tree, ok);
+      ok_all &= ok;
+      valid &= ok;
+      sK[row * LD + c] = valid ? (from_tree ? kt : kc)[off + c] : 0.f;
+      sV[row * LD + c] = valid ? (from_tree ? vt : vc)[off + c] : 0.f;
+    }
+    if (!ok_all) s_err = 1;
+    __syncthreads();
+    const bool tree_tile = t >= v.nPT;
+    const int kbase = tree_tile ? (t - v.nPT) * BN : t * BN;
+    const int lim = tree_tile ? v.N : v.L;
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) {
+      const int lr = warp * RPW + rr, r = r0 + lr;
+      if (r >= r_hi) continue;
+      float s = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) s = fmaf(sQ[lr * D + c], sK[lane * LD + c], s);
+      bool valid = kbase + lane < lim;
+      if (tree_tile && valid) {
+        const int node = r / G - i_lo, j = kbase + lane;
+        valid = (sMask[node * W + (j >> 5)] >> (j & 31)) & 1u;
+      }
+      s = valid ? s * sl2 : -INFINITY;
+      const float nm = fmaxf(m[rr], warp_max(s));
+      const float use = nm == -INFINITY ? 0.f : nm;
+      const float al = exp2f(m[rr] - use);
+      const float p = exp2f(s - use);
+      l[rr] = l[rr] * al + warp_sum(p);
+      m[rr] = nm;
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[rr][e] *= al;
+      for (int k = 0; k < BN; ++k) {
+        const float pk = __shfl_sync(0xffffffffu, p, k);
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[rr][e] = fmaf(pk, sV[k * LD + lane + 32 * e], o[rr][e]);
+      }
+    }
+  }
+  __syncthreads();
+  const bool err = s_err != 0;
+  if (err && split == 0 && mt == 0 && g == 0 && tid == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
+#pragma unroll
+  for (int rr = 0; rr < RPW; ++rr) {
+    const int r = r0 + warp * RPW + rr;
+    if (r >= r_hi) continue;
+    const int i = r / G, hh = r % G;
+    if (direct) {
+      float* out = reinterpret_cast<float*>(a.out) + (((size_t)b * a.Nmax + i) * a.Hq + g * G + hh) * D;
+      const float inv = (l[rr] > 0.f && !err) ? 1.f / l[rr] : 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) out[lane + 32 * e] = o[rr][e] * inv;
+      if (a.lse && lane == 0)
+        a.lse[((size_t)b * a.Nmax + i) * a.Hq + g * G + hh] = err ? 0.f : (m[rr] + __log2f(l[rr])) * kLn2;
+    } else {
+      float* wo = reinterpret_cast<float*>(a.workspace);
+      const size_t base = (((size_t)b * a.Hkv + g) * splits + split) * Rmax + r;
+      float* wml = wo + (size_t)a.B * a.Hkv * splits * Rmax * D;
+#pragma unroll
+      for (int e = 0; e < E; ++e) wo[base * D + lane + 32 * e] = o[rr][e];
+      if (lane == 0) *reinterpret_cast<float2*>(wml + base * 2) = make_float2(m[rr], l[rr]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Split merge: o = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), one warp per query row.
+// ------------------------------------------------------------------------------------------
+template <int D, typename OutT>
+__global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int splits, int Rmax) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int G = a.Hq / a.Hkv;
+  const SeqView v = seq_view(a, b, G, BN, tps);
+  if (v.skip || r >= v.R) return;
+  const int i = r / G, hh = r % G;
+  OutT* orow = reinterpret_cast<OutT*>(a.out) + (((size_t)b * a.Nmax + i) * a.Hq + g * G + hh) * D;
+  float* lrow = a.lse ? a.lse + ((size_t)b * a.Nmax + i) * a.Hq + g * G + hh : nullptr;
+  if (v.zero) {
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) store_out(orow + lane + 32 * e, 0.f);
+    if (lrow && lane == 0) *lrow = 0.f;
+    return;
+  }
+  if (v.nsplit <= 1) return;
+  const float* wo = reinterpret_cast<const float*>(a.workspace);
+  const float* wml = wo + (size_t)a.B * a.Hkv * splits * Rmax * D;
+  const size_t base = ((size_t)b * a.Hkv + g) * splits * Rmax + r;
+  float M = -INFINITY;
+  for (int s = 0; s < v.nsplit; ++s) M = fmaxf(M, wml[(base + (size_t)s * Rmax) * 2]);
+  const float Mu = M == -INFINITY ? 0.f : M;
+  float lsum = 0.f, acc[D / 32];
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+  for (int s = 0; s < v.nsplit; ++s) {
+    const size_t row = base + (size_t)s * Rmax;
+    const float2 ml = *reinterpret_cast<const float2*>(wml + row * 2);
+    const float w = exp2f(ml.x - Mu);
+    lsum += ml.y * w;
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(wo[row * D + lane + 32 * e], w, acc[e]);
+  }
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) store_out(orow + lane + 32 * e, acc[e] * inv);
+  if (lrow && lane == 0) *lrow = (M + __log2f(lsum)) * kLn2;
+}
+
+template <typename K>
+void set_smem_attr(K kernel, size_t bytes) {
+  // cheap and idempotent; needed once per kernel for > 48 KB of dynamic shared memory
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype) {
+  AttnPlan p;
+  p.G = Hq / Hkv;
+  p.Rmax = p.G * Nmax;
+  const int W = (Nmax + 31) / 32;
+  if (dtype == TSD_BF16) {
+    p.BN = 64;
+    p.BM = p.Rmax >= 128 ? 128 : ((p.Rmax + 15) / 16) * 16;
+    p.threads = p.BM / 16 * 32;
+    p.smem = (size_t)p.BM * d * 2 + (size_t)2 * kStages * p.BN * d * 2 + (size_t)(p.BM / p.G + 2) * W * 4;
+  } else {
+    p.BN = 32;
+    p.BM = 16;
+    p.threads = 128;
+    p.smem = (size_t)16 * d * 4 + (size_t)2 * 32 * (d + 1) * 4 + (size_t)(16 / p.G + 2) * W * 4;
+  }
+  if (p.BM <= 0) p.BM = 16;
+  p.mtiles = (p.Rmax + p.BM - 1) / p.BM;
+  p.max_tiles = (Lcap + p.BN - 1) / p.BN + (Nmax + p.BN - 1) / p.BN;
+  const long long base = (long long)B * Hkv * p.mtiles;
+  const int sms = device_sm_count();
+  const int want = base >= 2LL * sms ? 1 : (int)((2LL * sms + base - 1) / (base > 0 ? base : 1));
+  const int min_tps = (3 * p.BM / 2 + p.BN - 1) / p.BN;
+  int tps = (p.max_tiles + want - 1) / want;
+  if (tps < min_tps) tps = min_tps;
+  if (tps < 1) tps = 1;
+  if (tps > p.max_tiles) tps = p.max_tiles > 0 ? p.max_tiles : 1;
+  p.tps = tps;
+  p.splits = (p.max_tiles + tps - 1) / tps;
+  if (p.splits < 1) p.splits = 1;
+  p.ws_bytes = p.splits > 1 ? (size_t)B * Hkv * p.splits * p.Rmax * (d + 2) * sizeof(float) : 0;
+  return p;
+}
+
+tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream) {
+  if (a.B == 0 || a.Nmax == 0) return TSD_OK;
+  const AttnPlan p = plan_attention(a.B, a.Nmax, a.Hq, a.Hkv, a.d, a.Lcap, dtype);
+  dim3 grid(p.mtiles * p.splits, a.Hkv, a.B);
+  if (dtype == TSD_BF16) {
+    if (a.d == 128) {
+      set_smem_attr(attn_bf16_kernel<128>, p.smem);
+      attn_bf16_kernel<128><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
+    } else {
+      set_smem_attr(attn_bf16_kernel<64>, p.smem);
+      attn_bf16_kernel<64><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
+    }
+  } else {
+    if (a.d == 128) {
+      set_smem_attr(attn_f32_kernel<128>, p.smem);
+      attn_f32_kernel<128><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
+    } else {
+      set_smem_attr(attn_f32_kernel<64>, p.smem);
+      attn_f32_kernel<64><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
+    }
+  }
+  if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
+  if (p.splits > 1) {
+    const int rows_per_block = 8;
+    dim3 cg((p.Rmax + rows_per_block - 1) / rows_per_block, a.Hkv, a.B);
+    if (dtype == TSD_BF16) {
+      if (a.d == 128)
+        attn_combine_kernel<128, __nv_bfloat16><<<cg, 256, 0, stream>>>(a, p.BN, p.tps, p.splits, p.Rmax);
+      else
+        attn_combine_kernel<64, __nv_bfloat16><<<cg, 256, 0, stream>>>(a, p.BN, p.tps, p.splits, p.Rmax);
+    } else {
+      if (a.d == 128)
+        attn_combine_kernel<128, float><<<cg, 256, 0, stream>>>(a, p.BN, p.tps, p.splits, p.Rmax);
+      else
+        attn_combine_kernel<64, float><<<cg, 256, 0, stream>>>(a, p.BN, p.tps, p.splits, p.Rmax);
+    }
+    if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
+  }
+  return TSD_OK;
+}
+
+}  // namespace tsd

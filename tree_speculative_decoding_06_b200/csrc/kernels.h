@@ -1,0 +1,86 @@
+// Internal launch entry points of the kernels (host side); the C ABI in api.cu validates
+// arguments and calls these.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "tsd.h"
+
+namespace tsd {
+
+// Split-KV plan of one attention launch: a CTA covers BM query rows of one (sequence, KV head)
+// and `tps` key tiles of BN keys; the keys of sequence b are its prefix tiles followed by its
+// tree tiles.  Partials of (max, sum, unnormalised output) go to the workspace when a sequence
+// needs more than one split.
+struct AttnPlan {
+  int G = 1, Rmax = 0;      // query rows per (sequence, KV head) = G * Nmax
+  int BM = 0, mtiles = 0;   // rows per CTA, row tiles
+  int BN = 64;              // keys per tile
+  int max_tiles = 0;        // prefix tiles at capacity + tree tiles
+  int tps = 1, splits = 1;  // tiles per split, splits per (sequence, KV head, row tile)
+  int threads = 128;
+  size_t smem = 0;
+  size_t ws_bytes = 0;
+};
+
+struct AttnArgs {
+  const void* q;
+  const void* k_cache;      // contiguous [B,Hkv,Lmax,d] or pages [num_blocks,Hkv,bs,d]
+  const void* v_cache;
+  const int32_t* block_table;  // null = contiguous
+  int max_blocks, block_shift, num_blocks;
+  int Lcap;                 // Lmax or max_blocks * bs
+  const int32_t* prefix_len;
+  const void* k_tree;       // null = tree rows in the cache after the prefix
+  const void* v_tree;
+  const int32_t* parent_s;
+  const int32_t* num_nodes;
+  int B, Nmax, Hq, Hkv, d, Dmax;
+  float scale;
+  void* out;
+  float* lse;
+  void* workspace;
+  int32_t* status;
+};
+
+AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype);
+tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream);
+
+tsd_status launch_tree_prepare(const int32_t* parent, const int32_t* num_nodes, int B, int Nmax, int Dmax,
+                               int forest, int32_t* parent_s, int32_t* depth, int32_t* anc, uint32_t* anc_bits,
+                               int32_t* status, cudaStream_t stream);
+
+size_t accept_greedy_ws(int B, int Nmax, int V);
+tsd_status launch_accept_greedy(const void* logits, tsd_dtype dtype, int V, const int32_t* tokens,
+                                const int32_t* parent_s, const int32_t* num_nodes, const int32_t* root_key, int B,
+                                int Nmax, int Dmax, int32_t* accept_len, int32_t* path, int32_t* out_tokens,
+                                void* ws, int32_t* status, cudaStream_t stream);
+
+size_t chain_sample_ws(int B, int K, int V);
+tsd_status launch_chain_sample(const void* zp, const void* zq, tsd_dtype dtype, int V, const int32_t* x,
+                               const float* u, float T, int B, int K, int32_t* accept_len, int32_t* out_tokens,
+                               void* ws, cudaStream_t stream);
+
+struct CommitArgs {
+  void* k_cache;
+  void* v_cache;
+  const int32_t* block_table;  // null = contiguous [B,Hkv,Lmax,d]
+  int max_blocks, block_shift, num_blocks;
+  int Lcap;
+  int32_t* prefix_len;
+  const void* k_tree;
+  const void* v_tree;
+  const int32_t* path;
+  const int32_t* accept_len;
+  const int32_t* num_nodes;
+  int B, Nmax, Hkv, d, Dmax, esize;
+  int mode;
+  int32_t* status;
+};
+tsd_status launch_kv_commit(const CommitArgs& a, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace tsd
