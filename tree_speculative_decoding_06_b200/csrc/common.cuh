@@ -47,4 +47,22 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Load 8 consecutive logits starting at element `v` of a row (v % 8 == 0, 16-byte aligned row).
+template <typename T>
+__device__ __forceinline__ void load8(const T* row, int v, float (&x)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* row, int v, float (&x)[8]) {
+  const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + v));
+  x[0] = bf16_lo(w.x), x[1] = bf16_hi(w.x), x[2] = bf16_lo(w.y), x[3] = bf16_hi(w.y);
+  x[4] = bf16_lo(w.z), x[5] = bf16_hi(w.z), x[6] = bf16_lo(w.w), x[7] = bf16_hi(w.w);
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* row, int v, float (&x)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(row + v));
+  const float4 c = __ldg(reinterpret_cast<const float4*>(row + v + 4));
+  x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = c.x, x[5] = c.y, x[6] = c.z, x[7] = c.w;
+}
+__device__ __forceinline__ float load1(const __nv_bfloat16* row, int v) { return __bfloat162float(row[v]); }
+__device__ __forceinline__ float load1(const float* row, int v) { return row[v]; }
+
 }  // namespace tsd
