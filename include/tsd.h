@@ -201,6 +201,31 @@ tsd_status tsd_tree_accept_greedy(const void *logits, tsd_dtype dtype, int V, co
                                   void *stream);
 
 /* ---------------------------------------------------------------------------------------
+ * tsd_tree_accept_greedy_noalloc -- tsd_tree_accept_greedy for callers that cannot allocate.
+ * The pages have no counterpart of this call; it exists for library users whose code may not
+ * call cudaMalloc: a serving engine that gave all free device memory to its KV-cache pool at
+ * start-up, or a plug-in that a host runtime hands device pointers but no allocator.
+ *
+ * Same arguments, outputs and results as tsd_tree_accept_greedy, without the workspace: the
+ * scratch is a fixed array of TSD_ACCEPT_NOALLOC_SCRATCH_BYTES inside the library, present on
+ * every device that loads it until the process exits.  The call allocates nothing.
+ *   - A batch whose scratch need, tsd_tree_accept_greedy_workspace_size(B, Nmax, V), exceeds
+ *     TSD_ACCEPT_NOALLOC_SCRATCH_BYTES is refused with TSD_ERR_WORKSPACE before any launch
+ *     (1 MiB holds e.g. B*Nmax = 8192 rows of a 128256-token vocabulary).
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU (other streams, other
+ *     host threads) race and must be serialised by the caller.
+ * --------------------------------------------------------------------------------------- */
+#define TSD_ACCEPT_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+tsd_status tsd_tree_accept_greedy_noalloc(const void *logits, tsd_dtype dtype, int V, const int32_t *tokens,
+                                          const int32_t *parent_s, const int32_t *num_nodes,
+                                          const int32_t *root_key, int B, int Nmax, int Dmax,
+                                          int32_t *accept_len, int32_t *path, int32_t *out_tokens,
+                                          int32_t *status, void *stream);
+
+/* ---------------------------------------------------------------------------------------
  * tsd_chain_accept_sample -- rejection sampling of a linear draft of K tokens
  * ([SO] "Objetivo-Borrador": acceptance compares the full draft and target distributions and
  * the target's logits after the accepted run are sampled for one more token; the rule is the

@@ -43,6 +43,7 @@ _SIGS = {
                                         _I, _F, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_accept_greedy_workspace_size": (_SZ, [_I, _I, _I]),
     "tsd_tree_accept_greedy": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
+    "tsd_tree_accept_greedy_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "tsd_chain_accept_sample_workspace_size": (_SZ, [_I, _I, _I]),
     "tsd_chain_accept_sample": (_I, [_P, _P, _I, _I, _P, _P, _F, _I, _I, _P, _P, _P, _SZ, _P]),
     "tsd_kv_commit": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -216,6 +217,29 @@ def tree_accept_greedy(logits, tokens, parent_s, num_nodes=None, root_key=None, 
                                       _i32(root_key, "root_key"), B, Nmax, Dmax, _ptr(accept_len), _ptr(path),
                                       _ptr(out_tokens), _ptr(workspace), nbytes, _ptr(status), _stream(stream))
     _check(rc, "tsd_tree_accept_greedy")
+    return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
+
+
+ACCEPT_NOALLOC_SCRATCH_BYTES = 1 << 20
+
+
+def tree_accept_greedy_noalloc(logits, tokens, parent_s, num_nodes=None, root_key=None, Dmax: int = 8,
+                               accept_len=None, path=None, out_tokens=None, status=None, stream=None):
+    """tree_accept_greedy for callers that may not allocate device scratch: the library's own
+    fixed scratch array (ACCEPT_NOALLOC_SCRATCH_BYTES per device) is used instead of a
+    workspace.  Calls that overlap on the GPU share that array and race; the first call on a
+    device should come before any stream capture."""
+    B, Nmax, V = logits.shape
+    accept_len = _empty((B,), torch.int32, logits) if accept_len is None else accept_len
+    path = _empty((B, Dmax + 1), torch.int32, logits) if path is None else path
+    out_tokens = _empty((B, Dmax + 1), torch.int32, logits) if out_tokens is None else out_tokens
+    if status is None:
+        status = torch.zeros(B, dtype=torch.int32, device=logits.device)
+    rc = lib().tsd_tree_accept_greedy_noalloc(_ptr(logits), _dt(logits), V, _i32(tokens, "tokens"),
+                                              _i32(parent_s, "parent_s"), _i32(num_nodes, "num_nodes"),
+                                              _i32(root_key, "root_key"), B, Nmax, Dmax, _ptr(accept_len),
+                                              _ptr(path), _ptr(out_tokens), _ptr(status), _stream(stream))
+    _check(rc, "tsd_tree_accept_greedy_noalloc")
     return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
 
 

@@ -12,6 +12,7 @@
 // kChunk tokens over many CTAs (16-byte loads), and small per-sequence kernels merge the chunk
 // results.
 #include <climits>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -234,6 +235,42 @@ tsd_status launch_chain_sample(const void* zp, const void* zq, tsd_dtype dtype, 
                                                             nullptr, chunks, part);
   chain_greedy_decide<<<(B + 127) / 128, 128, 0, stream>>>(part, chunks, x, B, K, accept_len, out_tokens);
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// tsd_tree_accept_greedy_noalloc: the same acceptance with its scratch in a fixed device array.
+//
+// Some callers cannot allocate device memory for scratch: a serving engine that handed all free
+// device memory to its KV-cache pool at start-up, or a plug-in that a host runtime gives device
+// pointers but no allocator.  This variant needs no workspace argument: the argmax partials live
+// in g_accept_scratch, a file-scope array that every device loading this library holds until the
+// process exits.  Host code cannot pass the array's name to a kernel (in host code it names a
+// host-side stand-in), so the device address is fetched once per device with
+// cudaGetSymbolAddress, with that device current, on the first call made on it, and cached.
+// All calls share the array and it keeps the previous call's contents; nothing in it needs to
+// start at zero, because every entry the final kernel reads is written earlier in the same call.
+// Calls that overlap on the GPU (two streams, or two host threads) race on the array.
+// ---------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_accept_scratch[TSD_ACCEPT_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
+tsd_status accept_noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TSD_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_accept_scratch) != cudaSuccess || p == nullptr) return TSD_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return TSD_OK;
 }
 
 }  // namespace tsd

@@ -146,6 +146,26 @@ tsd_status tsd_tree_accept_greedy(const void* logits, tsd_dtype dtype, int V, co
                               path, out_tokens, workspace, status, S(stream));
 }
 
+tsd_status tsd_tree_accept_greedy_noalloc(const void* logits, tsd_dtype dtype, int V, const int32_t* tokens,
+                                          const int32_t* parent_s, const int32_t* num_nodes,
+                                          const int32_t* root_key, int B, int Nmax, int Dmax,
+                                          int32_t* accept_len, int32_t* path, int32_t* out_tokens, int32_t* status,
+                                          void* stream) {
+  if (!dtype_ok(dtype)) return TSD_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || B > 65535 || Nmax < 0 || Nmax > 65535 || V <= 0 || Dmax < 0 || Dmax > 255) return TSD_ERR_INVALID_ARG;
+  if ((long long)Nmax * 4 > 200 * 1024) return TSD_ERR_INVALID_ARG;
+  if (B == 0) return TSD_OK;
+  if (!accept_len || !path || !out_tokens || !status || !parent_s || (Nmax > 0 && (!logits || !tokens)))
+    return TSD_ERR_INVALID_ARG;
+  const size_t need = tsd_tree_accept_greedy_workspace_size(B, Nmax, V);
+  if (need > (size_t)TSD_ACCEPT_NOALLOC_SCRATCH_BYTES) return TSD_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const tsd_status e = accept_noalloc_scratch(&scratch);
+  if (e != TSD_OK) return e;
+  return launch_accept_greedy(logits, dtype, V, tokens, parent_s, num_nodes, root_key, B, Nmax, Dmax, accept_len,
+                              path, out_tokens, scratch, status, S(stream));
+}
+
 size_t tsd_chain_accept_sample_workspace_size(int B, int K, int V) {
   if (B <= 0 || K < 0 || V <= 0) return 0;
   return chain_sample_ws(B, K, V);

@@ -58,6 +58,8 @@ tsd_status launch_accept_greedy(const void* logits, tsd_dtype dtype, int V, cons
                                 int Nmax, int Dmax, int32_t* accept_len, int32_t* path, int32_t* out_tokens,
                                 void* ws, int32_t* status, cudaStream_t stream);
 
+tsd_status accept_noalloc_scratch(void** out);
+
 size_t chain_sample_ws(int B, int K, int V);
 tsd_status launch_chain_sample_stochastic(const void* zp, const void* zq, tsd_dtype dtype, int V, const int32_t* x,
                                           const float* u, float T, int B, int K, int32_t* accept_len,
