@@ -81,8 +81,19 @@ SMALL = {
 }
 
 
+@pytest.fixture(params=["auto", "mma"])
+def attn_path(request, monkeypatch):
+    """Run a test on the default kernel choice (tcgen05 where it applies) and again with the
+    warp-level mma.sync kernel forced, so both bf16 kernels stay covered."""
+    if request.param == "mma":
+        monkeypatch.setenv("TSD_ATTN_PATH", "mma")
+    else:
+        monkeypatch.delenv("TSD_ATTN_PATH", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("name", list(SMALL))
-def test_attention_small(name):
+def test_attention_small(name, attn_path):
     inp = W.make_inputs(SMALL[name])
     out, lse, st = gpu_attention(inp)
     assert (st == 0).all()
@@ -99,9 +110,9 @@ def test_attention_tree_in_cache(name):
 
 @pytest.mark.parametrize("dtype,d,Hq,Hkv,paged", [
     ("bf16", 64, 6, 2, False), ("bf16", 128, 5, 5, True), ("f32", 128, 12, 4, True), ("f32", 64, 3, 1, False),
-    ("bf16", 64, 48, 1, False),
+    ("bf16", 64, 48, 1, False), ("bf16", 128, 8, 8, True), ("bf16", 128, 64, 1, False), ("bf16", 128, 16, 2, True),
 ])
-def test_attention_shapes_and_ragged(dtype, d, Hq, Hkv, paged):
+def test_attention_shapes_and_ragged(dtype, d, Hq, Hkv, paged, attn_path):
     # ragged batch: empty prefix, a prefix that ends mid-tile, a long one; trees of different sizes
     parents = [W.tree_chain(1), W.tree_static_scored((4, 3, 2, 1, 1, 1), 26), W.tree_tiny(), W.tree_chain(70)]
     inp = W.make_custom_inputs(parents, [0, 63, 200, 129], Hq=Hq, Hkv=Hkv, d=d, dtype=dtype, seed=7, paged=paged,
@@ -153,7 +164,7 @@ FULL = ["tree26", "eagle60", "chain5", "forest"]
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_attention_full_size_sampled(name):
+def test_attention_full_size_sampled(name, attn_path):
     w = W.WORKLOADS[name]
     inp = W.make_inputs(w)
     out, lse, st = gpu_attention(inp)

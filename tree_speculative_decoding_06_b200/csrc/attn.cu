@@ -17,13 +17,17 @@
 // combine kernel merges by log-sum-exp.
 #include <climits>
 #include <cstdio>
+#include <cstdlib>
 
+#include "attn_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
 namespace tsd {
 
 namespace {
+
+using namespace attn;
 
 constexpr int kStages = 3;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -49,99 +53,6 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint
       "{%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Per-CTA view of one sequence: lengths, tile ranges and the early-exit verdicts.
-struct SeqView {
-  int N, R, L, nPT, T, nsplit;
-  bool skip, zero;   // skip: nothing to do; zero: write zeros (flagged / out of capacity)
-};
-
-__device__ __forceinline__ SeqView seq_view(const AttnArgs& a, int b, int G, int BN, int tps) {
-  SeqView v;
-  v.N = a.num_nodes ? a.num_nodes[b] : a.Nmax;
-  v.skip = (v.N <= 0 || v.N > a.Nmax);
-  v.R = G * v.N;
-  v.L = a.prefix_len[b];
-  const bool in_cache = (a.k_tree == nullptr);
-  const bool cap_bad = (v.L < 0) || ((long long)v.L + (in_cache ? v.N : 0) > a.Lcap);
-  v.zero = cap_bad || (a.status[b] != 0);
-  v.nPT = cap_bad ? 0 : (v.L + BN - 1) / BN;
-  v.T = v.nPT + (v.N + BN - 1) / BN;
-  v.nsplit = (v.T + tps - 1) / tps;
-  return v;
-}
-
-// Element offset of cache row `pos` of KV head g of sequence b; ok=false on a bad block id.
-__device__ __forceinline__ size_t cache_row(const AttnArgs& a, int b, int g, int pos, bool& ok) {
-  if (a.block_table == nullptr) return (((size_t)b * a.Hkv + g) * a.Lcap + pos) * a.d;
-  int blk = a.block_table[(size_t)b * a.max_blocks + (pos >> a.block_shift)];
-  if (blk < 0 || blk >= a.num_blocks) {
-    ok = false;
-    blk = 0;
-  }
-  const int off = pos & ((1 << a.block_shift) - 1);
-  return ((((size_t)blk * a.Hkv + g) << a.block_shift) + off) * a.d;
-}
-
-// Element offset (into k/v_cache or k/v_tree) of key `c` of tile t; sets from_tree.
-__device__ __forceinline__ size_t key_row(const AttnArgs& a, const SeqView& v, int b, int g, int t, int BN,
-                                          int c, bool& valid, bool& from_tree, bool& ok) {
-  if (t < v.nPT) {
-    const int k = t * BN + c;
-    valid = k < v.L;
-    from_tree = false;
-    return valid ? cache_row(a, b, g, k, ok) : 0;
-  }
-  const int j = (t - v.nPT) * BN + c;
-  valid = j < v.N;
-  if (a.k_tree == nullptr) {
-    from_tree = false;
-    return valid ? cache_row(a, b, g, v.L + j, ok) : 0;
-  }
-  from_tree = true;
-  return valid ? (((size_t)b * a.Nmax + j) * a.Hkv + g) * a.d : 0;
-}
-
-// Ancestor bits of the CTA's nodes i_lo..i_lo+cnt-1 over tree nodes, one row of W words each.
-__device__ __forceinline__ void build_mask(const AttnArgs& a, int b, int i_lo, int cnt, int W, uint32_t* smask) {
-  const int32_t* ps = a.parent_s + (size_t)b * (a.Nmax + 1);
-  for (int n = threadIdx.x; n < cnt; n += blockDim.x) {
-    uint32_t* row = smask + (size_t)n * W;
-    for (int w = 0; w < W; ++w) row[w] = 0u;
-    int s = i_lo + n + 1;
-    for (int step = 0; step <= a.Dmax && s != 0; ++step) {
-      const int j = s - 1;
-      row[j >> 5] |= 1u << (j & 31);
-      const int p = ps[s];
-      if (p >= s || p < 0) break;   // prepare rejects such trees; never walk upward-out-of-range
-      s = p;
-    }
-  }
-}
-
-template <typename OutT>
-__device__ __forceinline__ void store_out(OutT* o, float v);
-template <>
-__device__ __forceinline__ void store_out<float>(float* o, float v) { *o = v; }
-template <>
-__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* o, float v) { *o = __float2bfloat16_rn(v); }
-
-// Zero the output (and lse) rows [r_lo, r_hi) of (b, g).
-template <typename OutT>
-__device__ void zero_rows(const AttnArgs& a, int b, int g, int G, int r_lo, int r_hi) {
-  OutT* out = reinterpret_cast<OutT*>(a.out);
-  const int D = a.d;
-  for (int idx = threadIdx.x; idx < (r_hi - r_lo) * D; idx += blockDim.x) {
-    const int r = r_lo + idx / D, c = idx % D;
-    const int i = r / G, hh = r % G;
-    store_out(out + (((size_t)b * a.Nmax + i) * a.Hq + g * G + hh) * D + c, 0.f);
-  }
-  if (a.lse)
-    for (int r = r_lo + threadIdx.x; r < r_hi; r += blockDim.x) {
-      const int i = r / G, hh = r % G;
-      a.lse[((size_t)b * a.Nmax + i) * a.Hq + g * G + hh] = 0.f;
-    }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -219,7 +130,7 @@ __global__ void __launch_bounds__(256, 1)
     if (s < nt) load_tile(t_begin + s, s);
     cp_async_commit();
   }
-  if (t_end > v.nPT) build_mask(a, b, i_lo, i_cnt, W, sMask);
+  if (t_end > v.nPT) build_mask(a, b, i_lo, i_cnt, W, sMask, v.N);
 
   // per-thread rows: A = lane/4, B = lane/4 + 8 of this warp's 16
   const int wr0 = r0 + warp * 16;
@@ -432,7 +343,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a, int BM,
     if (r < v.R) x = q[(((size_t)b * a.Nmax + r / G) * a.Hq + g * G + r % G) * D + c];
     sQ[row * D + c] = x;
   }
-  if (t_end > v.nPT) build_mask(a, b, i_lo, i_cnt, W, sMask);
+  if (t_end > v.nPT) build_mask(a, b, i_lo, i_cnt, W, sMask, v.N);
   const float sl2 = a.scale * kLog2e;
   float m[RPW], l[RPW], o[RPW][E];
 #pragma unroll
@@ -537,20 +448,35 @@ __global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int split
   const float* wo = reinterpret_cast<const float*>(a.workspace);
   const float* wml = wo + (size_t)a.B * a.Hkv * splits * Rmax * D;
   const size_t base = ((size_t)b * a.Hkv + g) * splits * Rmax + r;
+  // lane s holds split s's (max, sum): all of them are fetched at once, not one after another
   float M = -INFINITY;
-  for (int s = 0; s < v.nsplit; ++s) M = fmaxf(M, wml[(base + (size_t)s * Rmax) * 2]);
+  for (int s0 = 0; s0 < v.nsplit; s0 += 32) {
+    const int s = s0 + lane;
+    if (s < v.nsplit) M = fmaxf(M, wml[(base + (size_t)s * Rmax) * 2]);
+  }
+  M = warp_max(M);
   const float Mu = M == -INFINITY ? 0.f : M;
   float lsum = 0.f, acc[D / 32];
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
-  for (int s = 0; s < v.nsplit; ++s) {
-    const size_t row = base + (size_t)s * Rmax;
-    const float2 ml = *reinterpret_cast<const float2*>(wml + row * 2);
-    const float w = exp2f(ml.x - Mu);
-    lsum += ml.y * w;
+  for (int s0 = 0; s0 < v.nsplit; s0 += 32) {
+    const int s = s0 + lane;
+    float w = 0.f;
+    if (s < v.nsplit) {
+      const float2 ml = *reinterpret_cast<const float2*>(wml + (base + (size_t)s * Rmax) * 2);
+      w = exp2f(ml.x - Mu);
+      lsum += ml.y * w;
+    }
+    const int n = min(32, v.nsplit - s0);
+#pragma unroll 4
+    for (int k = 0; k < n; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, k);
+      const float* src = wo + (base + (size_t)(s0 + k) * Rmax) * D + lane;
 #pragma unroll
-    for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(wo[row * D + lane + 32 * e], w, acc[e]);
+      for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(src[32 * e], wk, acc[e]);
+    }
   }
+  lsum = warp_sum(lsum);
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) store_out(orow + lane + 32 * e, acc[e] * inv);
@@ -609,7 +535,13 @@ tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t str
   if (a.B == 0 || a.Nmax == 0) return TSD_OK;
   const AttnPlan p = plan_attention(a.B, a.Nmax, a.Hq, a.Hkv, a.d, a.Lcap, dtype);
   dim3 grid(p.mtiles * p.splits, a.Hkv, a.B);
-  if (dtype == TSD_BF16) {
+  // TSD_ATTN_PATH=mma selects the warp-level kernel even where the tcgen05 kernel applies (A/B runs)
+  const char* path_env = getenv("TSD_ATTN_PATH");
+  const bool force_mma = path_env != nullptr && path_env[0] == 'm' && path_env[1] == 'm';
+  if (dtype == TSD_BF16 && !force_mma && umma_eligible(a, dtype)) {
+    const tsd_status st = launch_attention_umma(a, p, stream);
+    if (st != TSD_OK) return st;
+  } else if (dtype == TSD_BF16) {
     if (a.d == 128) {
       set_smem_attr(attn_bf16_kernel<128>, p.smem);
       attn_bf16_kernel<128><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);

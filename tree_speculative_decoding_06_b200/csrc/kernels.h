@@ -47,6 +47,9 @@ struct AttnArgs {
 
 AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype);
 tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream);
+// tcgen05 path (attn_umma.cu): bf16, d = 128, tree K/V in their own buffer, G a power of two.
+bool umma_eligible(const AttnArgs& a, tsd_dtype dtype);
+tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStream_t stream);
 
 tsd_status launch_tree_prepare(const int32_t* parent, const int32_t* num_nodes, int B, int Nmax, int Dmax,
                                int forest, int32_t* parent_s, int32_t* depth, int32_t* anc, uint32_t* anc_bits,
