@@ -53,14 +53,19 @@ __device__ __forceinline__ void block_argmax(float& bv, int& bi) {
 }
 
 // Argmax of one chunk of one row.  rows_per_seq rows per sequence; row i >= n_b is skipped.
+// The scan reads only the logits (inputs), so it runs before pdl_wait(); the partial is written
+// after it (the previous step's acceptance may still be reading the workspace).
 template <typename T>
 __global__ void __launch_bounds__(kThreads) row_argmax_chunks(const T* __restrict__ logits, int V, int rows_per_seq,
-                                                              const int32_t* __restrict__ num_rows,
-                                                              const int32_t* __restrict__ status, int chunks,
+                                                              const int32_t* __restrict__ num_rows, int chunks,
                                                               float2* __restrict__ part) {
+  pdl_trigger();
   const int c = blockIdx.x, i = blockIdx.y, b = blockIdx.z;
   const int n = num_rows ? num_rows[b] : rows_per_seq;
-  if (i >= n || (status && status[b] != 0)) return;
+  if (i >= n) {
+    pdl_wait();
+    return;
+  }
   const T* row = logits + ((size_t)b * rows_per_seq + i) * V;
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
   float bv = -INFINITY;
@@ -80,6 +85,7 @@ __global__ void __launch_bounds__(kThreads) row_argmax_chunks(const T* __restric
     }
   }
   block_argmax(bv, bi);
+  pdl_wait();
   if (threadIdx.x == 0) {
     if (bv == -INFINITY || bi == INT_MAX) bi = lo;   // nothing above -inf: the chunk's first index
     part[((size_t)b * rows_per_seq + i) * chunks + c] = make_float2(bv, __int_as_float(bi));
@@ -107,6 +113,8 @@ __global__ void __launch_bounds__(kThreads) tree_accept_kernel(const float2* __r
                                                                int32_t* __restrict__ path,
                                                                int32_t* __restrict__ out_tokens,
                                                                const int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int32_t s_tstar[];
   __shared__ int s_hit, s_best;
   const int b = blockIdx.x;
@@ -171,6 +179,8 @@ __global__ void __launch_bounds__(kThreads) tree_accept_kernel(const float2* __r
 __global__ void chain_greedy_decide(const float2* __restrict__ part, int chunks, const int32_t* __restrict__ x,
                                     int B, int K, int32_t* __restrict__ accept_len,
                                     int32_t* __restrict__ out_tokens) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= B) return;
   int j = K;
@@ -202,18 +212,18 @@ tsd_status launch_accept_greedy(const void* logits, tsd_dtype dtype, int V, cons
   if (Nmax > 0) {
     dim3 grid(chunks, Nmax, B);
     if (dtype == TSD_BF16)
-      row_argmax_chunks<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
-          reinterpret_cast<const __nv_bfloat16*>(logits), V, Nmax, num_nodes, status, chunks, part);
+      launch_pdl(row_argmax_chunks<__nv_bfloat16>, grid, dim3(kThreads), 0, stream,
+                 reinterpret_cast<const __nv_bfloat16*>(logits), V, Nmax, num_nodes, chunks, part);
     else
-      row_argmax_chunks<float><<<grid, kThreads, 0, stream>>>(reinterpret_cast<const float*>(logits), V, Nmax,
-                                                              num_nodes, status, chunks, part);
+      launch_pdl(row_argmax_chunks<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(logits), V,
+                 Nmax, num_nodes, chunks, part);
     if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
   }
   const size_t smem = (size_t)(Nmax > 0 ? Nmax : 1) * sizeof(int32_t);
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(tree_accept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  tree_accept_kernel<<<B, kThreads, smem, stream>>>(part, chunks, tokens, parent_s, num_nodes, root_key, Nmax, Dmax,
-                                                    accept_len, path, out_tokens, status);
+  launch_pdl(tree_accept_kernel, dim3(B), dim3(kThreads), smem, stream, (const float2*)part, chunks, tokens, parent_s,
+             num_nodes, root_key, Nmax, Dmax, accept_len, path, out_tokens, (const int32_t*)status);
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }
 
@@ -228,12 +238,13 @@ tsd_status launch_chain_sample(const void* zp, const void* zq, tsd_dtype dtype, 
   float2* part = reinterpret_cast<float2*>(ws);
   dim3 grid(chunks, K + 1, B);
   if (dtype == TSD_BF16)
-    row_argmax_chunks<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(zp), V,
-                                                                    K + 1, nullptr, nullptr, chunks, part);
+    launch_pdl(row_argmax_chunks<__nv_bfloat16>, grid, dim3(kThreads), 0, stream,
+               reinterpret_cast<const __nv_bfloat16*>(zp), V, K + 1, (const int32_t*)nullptr, chunks, part);
   else
-    row_argmax_chunks<float><<<grid, kThreads, 0, stream>>>(reinterpret_cast<const float*>(zp), V, K + 1, nullptr,
-                                                            nullptr, chunks, part);
-  chain_greedy_decide<<<(B + 127) / 128, 128, 0, stream>>>(part, chunks, x, B, K, accept_len, out_tokens);
+    launch_pdl(row_argmax_chunks<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(zp), V, K + 1,
+               (const int32_t*)nullptr, chunks, part);
+  launch_pdl(chain_greedy_decide, dim3((B + 127) / 128), dim3(128), 0, stream, (const float2*)part, chunks, x, B, K,
+             accept_len, out_tokens);
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }
 

@@ -62,6 +62,8 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint
 template <int D>
 __global__ void __launch_bounds__(256, 1)
     attn_bf16_kernel(const AttnArgs a, int BM, int mtiles, int tps, int splits, int Rmax) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int BN = 64;
   constexpr int CH = D / 8;   // 16-byte chunks per row
   extern __shared__ __align__(128) uint8_t smem[];
@@ -306,6 +308,8 @@ __global__ void __launch_bounds__(256, 1)
 template <int D>
 __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a, int BM, int mtiles, int tps, int splits,
                                                        int Rmax) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int BN = 32, RPW = 4, E = D / 32, LD = D + 1;
   extern __shared__ __align__(128) uint8_t smem[];
   float* sQ = reinterpret_cast<float*>(smem);
@@ -429,6 +433,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a, int BM,
 // ------------------------------------------------------------------------------------------
 template <int D, typename OutT>
 __global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int splits, int Rmax) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * (blockDim.x >> 5) + warp;
   const int g = blockIdx.y, b = blockIdx.z;
@@ -544,18 +550,18 @@ tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t str
   } else if (dtype == TSD_BF16) {
     if (a.d == 128) {
       set_smem_attr(attn_bf16_kernel<128>, p.smem);
-      attn_bf16_kernel<128><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
+      launch_pdl(attn_bf16_kernel<128>, grid, dim3(p.threads), p.smem, stream, a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
     } else {
       set_smem_attr(attn_bf16_kernel<64>, p.smem);
-      attn_bf16_kernel<64><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
+      launch_pdl(attn_bf16_kernel<64>, grid, dim3(p.threads), p.smem, stream, a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
     }
   } else {
     if (a.d == 128) {
       set_smem_attr(attn_f32_kernel<128>, p.smem);
-      attn_f32_kernel<128><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
+      launch_pdl(attn_f32_kernel<128>, grid, dim3(p.threads), p.smem, stream, a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
     } else {
       set_smem_attr(attn_f32_kernel<64>, p.smem);
-      attn_f32_kernel<64><<<grid, p.threads, p.smem, stream>>>(a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
+      launch_pdl(attn_f32_kernel<64>, grid, dim3(p.threads), p.smem, stream, a, p.BM, p.mtiles, p.tps, p.splits, p.Rmax);
     }
   }
   if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
@@ -564,14 +570,14 @@ tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t str
     dim3 cg((p.Rmax + rows_per_block - 1) / rows_per_block, a.Hkv, a.B);
     if (dtype == TSD_BF16) {
       if (a.d == 128)
-        attn_combine_kernel<128, __nv_bfloat16><<<cg, 256, 0, stream>>>(a, p.BN, p.tps, p.splits, p.Rmax);
+        launch_pdl(attn_combine_kernel<128, __nv_bfloat16>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax);
       else
-        attn_combine_kernel<64, __nv_bfloat16><<<cg, 256, 0, stream>>>(a, p.BN, p.tps, p.splits, p.Rmax);
+        launch_pdl(attn_combine_kernel<64, __nv_bfloat16>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax);
     } else {
       if (a.d == 128)
-        attn_combine_kernel<128, float><<<cg, 256, 0, stream>>>(a, p.BN, p.tps, p.splits, p.Rmax);
+        launch_pdl(attn_combine_kernel<128, float>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax);
       else
-        attn_combine_kernel<64, float><<<cg, 256, 0, stream>>>(a, p.BN, p.tps, p.splits, p.Rmax);
+        launch_pdl(attn_combine_kernel<64, float>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax);
     }
     if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
   }

@@ -6,15 +6,19 @@
 // tree's keys), built for Blackwell:
 //   * a CTA owns 128 query rows (G heads x 128/G tree nodes of one KV head) and a range of 64-key
 //     tiles of one sequence; every K/V tile is read from memory once per 128 rows;
-//   * warp 0 streams the tiles with TMA (128-byte swizzled boxes; paged caches box by block, the
-//     tree's K/V by node for one KV head) through a 4-deep ring of shared-memory stages;
-//   * warp 1 issues tcgen05.mma from one thread: S = Q K^T into a double-buffered TMEM tile
-//     (128 lanes x 64 fp32 columns), then O += P V into a 128 x 128 fp32 TMEM accumulator;
-//   * warps 4-7 each own one TMEM lane quarter, one query row per thread: a row's 64 scores come
-//     out of TMEM with one tcgen05.ld, so its max and sum need no shuffles; the ancestor mask is
-//     applied only on tree tiles (bits rebuilt in shared memory by warps 2-3); P is written back
-//     as bf16 into a swizzled shared tile for the P V product.  The running max is raised
-//     lazily (only when a row's max grows by more than 2^8), so O is rescaled in TMEM rarely.
+//   * two producer threads stream K and V tiles with TMA (128-byte swizzled boxes; paged caches
+//     box by block, the tree's K/V by node for one KV head) into separate rings: a K slot is
+//     released as soon as S = Q K^T has read it, a V slot after P V, so loads run several tiles
+//     ahead of the math;
+//   * one thread issues tcgen05.mma: S into one of two TMEM tiles (128 lanes x 64 fp32 columns)
+//     and O += P V into one of two 128 x 128 fp32 TMEM accumulators;
+//   * two softmax warpgroups take alternate tiles (even / odd), each with its own S tile, P
+//     buffer, O accumulator and running (max, sum) -- a split of the key range inside the CTA,
+//     merged by log-sum-exp in the epilogue.  In a warpgroup each warp owns one TMEM lane
+//     quarter, one query row per thread: a row's 64 scores come out of TMEM with one tcgen05.ld,
+//     so its max and sum need no shuffles.  The ancestor mask is applied only on tree tiles (bits
+//     rebuilt in shared memory at set-up); full prefix tiles take a lean path (no mask work).  The
+//     running max is raised lazily (only past a 2^8 growth), so O is rescaled in TMEM rarely.
 // Every mbarrier wait is bounded: on time-out the CTA records TSD_ERR_TIMEOUT, drains its own
 // TMA copies (again bounded) and frees its TMEM before returning.
 #include <cuda.h>
@@ -36,34 +40,42 @@ using namespace attn;
 using namespace umma;
 
 constexpr int kBM = 128, kBN = 64, kD = 128;
-constexpr int kThreadsU = 256;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColO = 0, kColS = 128;        // S buffers at columns 128 and 192
+constexpr int kThreadsU = 384;                    // 12 warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0, kColS = 256;         // O_w at 128*w, S_w at 256 + 64*w
 constexpr uint32_t kHalf = kBN * 128;              // one 64-column half of a K or V tile: 8 KB
-constexpr uint32_t kStageBytes = 4 * kHalf;        // K halves + V halves: 32 KB
+constexpr uint32_t kSlot = 2 * kHalf;              // one K or V tile: 16 KB
 constexpr uint32_t kQBytes = kBM * 256;            // 32 KB
-constexpr uint32_t kPBytes = kBM * 128;            // 16 KB
+constexpr uint32_t kPBytes = kBM * 128;            // 16 KB per softmax warpgroup
+constexpr int kMaxRing = 6;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;               // lazy max: rescale only past a 2^8 growth
 
 struct UParams {
-  int tps, splits, Rmax, mtiles, stages;
+  int tps, splits, Rmax, mtiles;
+  int ks, vs;          // K and V ring depths
   int box_rows;        // rows per TMA box of the cache (64 contiguous, min(block, 64) paged)
   int W;               // ancestor-bit words per node
-  uint32_t mask_off;   // shared-memory offsets
-  uint32_t p_off;
+  uint32_t k_off, v_off, p_off, mask_off;   // shared-memory offsets
 };
 
 struct __align__(8) Bars {
   uint64_t q_full;
-  uint64_t s_full[2];
-  uint64_t p_full;
-  uint64_t pv_done;
-  uint64_t kv_full[4];
-  uint64_t kv_empty[4];
+  uint64_t k_full[kMaxRing], k_empty[kMaxRing];
+  uint64_t v_full[kMaxRing], v_empty[kMaxRing];
+  uint64_t s_full[2];    // warpgroup w: its S tile is in TMEM
+  uint64_t p_full[2];    // warpgroup w: its P tile is in shared memory (and its S tile was read)
+  uint64_t pv_done[2];   // warpgroup w: its last P V product finished (P buffer free, O current)
   uint64_t fin;
 };
+
+// 2^x with the hardware approximation (flush-to-zero; 2^-inf = 0).  P is rounded to bf16 anyway.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ void abort_cta(const AttnArgs& a, int b, volatile int* s_abort) {
   if (*s_abort == 0) {
@@ -72,17 +84,53 @@ __device__ __forceinline__ void abort_cta(const AttnArgs& a, int b, volatile int
   }
 }
 
+// TMA loads of one 64-key tile (K or V half pair) of sequence b, KV head g into `dst`.
+__device__ __forceinline__ void load_tile(const AttnArgs& a, const SeqView& v, const UParams& u, int b, int g,
+                                          int t, uint8_t* dst, const CUtensorMap* cache_map,
+                                          const CUtensorMap* tree_map, uint64_t* bar, int* s_err) {
+  if (t < v.nPT) {
+    const int pos0 = t * kBN;
+    if (a.block_table == nullptr) {
+      const int y = (b * a.Hkv + g) * a.Lcap + pos0;
+      tma_load_2d(dst, cache_map, 0, y, bar);
+      tma_load_2d(dst + kHalf, cache_map, 64, y, bar);
+    } else {
+      const int bs_mask = (1 << a.block_shift) - 1;
+      for (int seg = 0; seg < kBN; seg += u.box_rows) {
+        const int pos = pos0 + seg;
+        const int bi = min(pos >> a.block_shift, a.max_blocks - 1);
+        int blk = a.block_table[(size_t)b * a.max_blocks + bi];
+        if (blk < 0 || blk >= a.num_blocks) {
+          if (pos < v.L) *s_err = 1;
+          blk = 0;
+        }
+        const int y = (blk * a.Hkv + g) * (1 << a.block_shift) + (pos & bs_mask);
+        const uint32_t off = (uint32_t)seg * 128;
+        tma_load_2d(dst + off, cache_map, 0, y, bar);
+        tma_load_2d(dst + kHalf + off, cache_map, 64, y, bar);
+      }
+    }
+  } else {
+    const int z = b * a.Nmax + (t - v.nPT) * kBN;
+    tma_load_3d(dst, tree_map, 0, g, z, bar);
+    tma_load_3d(dst + kHalf, tree_map, 64, g, z, bar);
+  }
+}
+
 __global__ void __launch_bounds__(kThreadsU, 1)
     attn_umma_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
                      const __grid_constant__ CUtensorMap tmVt, const AttnArgs a, const UParams u) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ Bars bars;
   __shared__ uint32_t s_tmem;
   __shared__ int s_err;
   __shared__ volatile int s_abort;
-  __shared__ int s_issued, s_consumed;
+  __shared__ int s_k_issued, s_v_issued, s_k_consumed, s_v_consumed;
+  __shared__ float2 s_ml1[kBM];   // warpgroup 1's (max, sum) per row, for the epilogue merge
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int mt = blockIdx.x % u.mtiles, split = blockIdx.x / u.mtiles;
@@ -105,26 +153,25 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   const int node0 = mt * nodes_per_tile;
 
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + kQBytes;
+  uint8_t* sK = smem + u.k_off;
+  uint8_t* sV = smem + u.v_off;
   uint8_t* sP = smem + u.p_off;
   uint32_t* sMask = reinterpret_cast<uint32_t*>(smem + u.mask_off);
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
     mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.s_full[0], 1);
-    mbar_init(&bars.s_full[1], 1);
-    mbar_init(&bars.p_full, 4);
-    mbar_init(&bars.pv_done, 1);
-    mbar_init(&bars.fin, 1);
-    for (int s = 0; s < u.stages; ++s) {
-      mbar_init(&bars.kv_full[s], 1);
-      mbar_init(&bars.kv_empty[s], 1);
+    for (int s = 0; s < u.ks; ++s) mbar_init(&bars.k_full[s], 1), mbar_init(&bars.k_empty[s], 1);
+    for (int s = 0; s < u.vs; ++s) mbar_init(&bars.v_full[s], 1), mbar_init(&bars.v_empty[s], 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bars.s_full[w], 1);
+      mbar_init(&bars.p_full[w], 4);
+      mbar_init(&bars.pv_done[w], 1);
     }
+    mbar_init(&bars.fin, 1);
     s_err = 0;
     s_abort = 0;
-    s_issued = 0;
-    s_consumed = 0;
+    s_k_issued = s_v_issued = s_k_consumed = s_v_consumed = 0;
     fence_barrier_init();
     fence_proxy_async();
   }
@@ -132,101 +179,65 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     tmem_alloc(&s_tmem, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 2 || warp == 3) {
-    if (t_begin + nt > v.nPT) build_mask(a, b, node0, nodes_per_tile, u.W, sMask, v.N, tid - 64, 64);
+  if (warp == 3) {
+    if (t_begin + nt > v.nPT) build_mask(a, b, node0, nodes_per_tile, u.W, sMask, v.N, lane, 32);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  float row_state_m = -INFINITY, row_state_l = 0.f;   // softmax threads: the row's final max and sum
+  float row_m = -INFINITY, row_l = 0.f;   // softmax threads: the row's final (max, sum) for their warpgroup
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (one thread)
+    // ------------------------------------------------------------ K producer (one thread), Q first
     if (lane == 0) {
       mbar_expect_tx(&bars.q_full, kQBytes);
       const int zq = b * a.Nmax + node0;
       tma_load_3d(sQ, &tmQ, 0, g * G, zq, &bars.q_full);
       tma_load_3d(sQ + kQBytes / 2, &tmQ, 64, g * G, zq, &bars.q_full);
       int issued = 0;
-      for (int i = 0; i < nt; ++i) {
-        const int st = i % u.stages;
-        if (i >= u.stages && !mbar_wait(&bars.kv_empty[st], ((i / u.stages) - 1) & 1)) {
+      for (int i = 0; i < nt && !s_abort; ++i) {
+        const int st = i % u.ks;
+        if (i >= u.ks && !mbar_wait(&bars.k_empty[st], ((i / u.ks) - 1) & 1)) {
           abort_cta(a, b, &s_abort);
           break;
         }
-        if (s_abort) break;
-        uint8_t* dK = sKV + (size_t)st * kStageBytes;
-        uint8_t* dV = dK + 2 * kHalf;
-        mbar_expect_tx(&bars.kv_full[st], kStageBytes);
-        const int t = t_begin + i;
-        if (t < v.nPT) {
-          const int pos0 = t * kBN;
-          if (a.block_table == nullptr) {
-            const int y = (b * a.Hkv + g) * a.Lcap + pos0;
-            tma_load_2d(dK, &tmK, 0, y, &bars.kv_full[st]);
-            tma_load_2d(dK + kHalf, &tmK, 64, y, &bars.kv_full[st]);
-            tma_load_2d(dV, &tmV, 0, y, &bars.kv_full[st]);
-            tma_load_2d(dV + kHalf, &tmV, 64, y, &bars.kv_full[st]);
-          } else {
-            const int bs_mask = (1 << a.block_shift) - 1;
-            for (int seg = 0; seg < kBN; seg += u.box_rows) {
-              const int pos = pos0 + seg;
-              const int bi = min(pos >> a.block_shift, a.max_blocks - 1);
-              int blk = a.block_table[(size_t)b * a.max_blocks + bi];
-              if (blk < 0 || blk >= a.num_blocks) {
-                if (pos < v.L) s_err = 1;
-                blk = 0;
-              }
-              const int y = (blk * a.Hkv + g) * (1 << a.block_shift) + (pos & bs_mask);
-              const uint32_t off = (uint32_t)seg * 128;
-              tma_load_2d(dK + off, &tmK, 0, y, &bars.kv_full[st]);
-              tma_load_2d(dK + kHalf + off, &tmK, 64, y, &bars.kv_full[st]);
-              tma_load_2d(dV + off, &tmV, 0, y, &bars.kv_full[st]);
-              tma_load_2d(dV + kHalf + off, &tmV, 64, y, &bars.kv_full[st]);
-            }
-          }
-        } else {
-          const int z = b * a.Nmax + (t - v.nPT) * kBN;
-          tma_load_3d(dK, &tmKt, 0, g, z, &bars.kv_full[st]);
-          tma_load_3d(dK + kHalf, &tmKt, 64, g, z, &bars.kv_full[st]);
-          tma_load_3d(dV, &tmVt, 0, g, z, &bars.kv_full[st]);
-          tma_load_3d(dV + kHalf, &tmVt, 64, g, z, &bars.kv_full[st]);
-        }
+        mbar_expect_tx(&bars.k_full[st], kSlot);
+        load_tile(a, v, u, b, g, t_begin + i, sK + (size_t)st * kSlot, &tmK, &tmKt, &bars.k_full[st], &s_err);
         ++issued;
       }
-      s_issued = issued;
+      s_k_issued = issued;
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ V producer (one thread)
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nt && !s_abort; ++i) {
+        const int st = i % u.vs;
+        if (i >= u.vs && !mbar_wait(&bars.v_empty[st], ((i / u.vs) - 1) & 1)) {
+          abort_cta(a, b, &s_abort);
+          break;
+        }
+        mbar_expect_tx(&bars.v_full[st], kSlot);
+        load_tile(a, v, u, b, g, t_begin + i, sV + (size_t)st * kSlot, &tmV, &tmVt, &bars.v_full[st], &s_err);
+        ++issued;
+      }
+      s_v_issued = issued;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (one thread)
     const uint32_t idesc_s = idesc_bf16(kBM, kBN, false);
     const uint32_t idesc_o = idesc_bf16(kBM, kD, true);
-    const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+    const uint32_t q_addr = smem_u32(sQ);
     bool ok = mbar_wait(&bars.q_full, 0);
-    int consumed = 0;
-    // zero V rows past the valid keys of a partial tile (its TMA box may hold stale rows)
-    auto ready_tile = [&](int i) -> bool {
-      const int st = i % u.stages;
-      if (!mbar_wait(&bars.kv_full[st], (i / u.stages) & 1)) return false;
-      ++consumed;
-      const int t = t_begin + i;
-      const int nv = t < v.nPT ? min(kBN, v.L - t * kBN) : min(kBN, v.N - (t - v.nPT) * kBN);
-      if (nv < kBN) {
-        uint8_t* dV = sKV + (size_t)st * kStageBytes + 2 * kHalf;
-        const int nchunks = (kBN - nv) * 8;   // 16-byte chunks per half
-        for (int c = lane; c < 2 * nchunks; c += 32) {
-          const int half = c / nchunks, cc = c % nchunks;
-          *reinterpret_cast<uint4*>(dV + half * kHalf + (size_t)nv * 128 + (size_t)cc * 16) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async();
-      }
-      __syncwarp();
-      return true;
-    };
-    auto issue_s = [&](int i) {
-      const int st = i % u.stages;
-      const uint32_t k_addr = smem_u32(sKV + (size_t)st * kStageBytes);
-      const uint32_t d = tmem + kColS + (uint32_t)(i & 1) * kBN;
+    int k_consumed = 0, v_consumed = 0;
+    // S(j) = Q K(j)^T into warpgroup (j & 1)'s S tile; frees the K slot when done
+    auto issue_s = [&](int j) -> bool {
+      const int st = j % u.ks;
+      if (!mbar_wait(&bars.k_full[st], (j / u.ks) & 1)) return false;
+      ++k_consumed;
+      const uint32_t k_addr = smem_u32(sK + (size_t)st * kSlot);
+      const uint32_t d = tmem + kColS + (uint32_t)(j & 1) * kBN;
       if (lane == 0) {
         tc_fence_after();
 #pragma unroll
@@ -236,199 +247,268 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           const uint64_t bd = sdesc_sw128(k_addr + half * kHalf + within, 16, 1024);
           mma_bf16_ss(d, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bars.s_full[i & 1]);
+        tc_commit(&bars.k_empty[st]);
+        tc_commit(&bars.s_full[j & 1]);
       }
       __syncwarp();
+      return true;
     };
-    if (ok && nt > 0) {
-      ok = ready_tile(0);
-      if (ok) issue_s(0);
-    }
+    if (ok && nt > 0) ok = issue_s(0);
+    if (ok && nt > 1) ok = issue_s(1);
     for (int i = 0; ok && i < nt; ++i) {
-      if (i + 1 < nt) {
-        ok = ready_tile(i + 1);
-        if (!ok) break;
-        issue_s(i + 1);
-      }
-      if (!mbar_wait(&bars.p_full, i & 1)) {
+      const int w = i & 1;
+      if (!mbar_wait(&bars.p_full[w], (i >> 1) & 1)) {
         ok = false;
         break;
       }
-      const int st = i % u.stages;
-      const uint32_t v_addr = smem_u32(sKV + (size_t)st * kStageBytes + 2 * kHalf);
+      const int st = i % u.vs;
+      if (!mbar_wait(&bars.v_full[st], (i / u.vs) & 1)) {
+        ok = false;
+        break;
+      }
+      ++v_consumed;
+      // zero V rows past the valid keys of a partial tile (its TMA box may hold stale rows)
+      const int t = t_begin + i;
+      const int nv = t < v.nPT ? min(kBN, v.L - t * kBN) : min(kBN, v.N - (t - v.nPT) * kBN);
+      uint8_t* dV = sV + (size_t)st * kSlot;
+      if (nv < kBN) {
+        const int nchunks = (kBN - nv) * 8;   // 16-byte chunks per half
+        for (int c = lane; c < 2 * nchunks; c += 32) {
+          const int half = c / nchunks, cc = c % nchunks;
+          *reinterpret_cast<uint4*>(dV + half * kHalf + (size_t)nv * 128 + (size_t)cc * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();
+      }
+      __syncwarp();
+      const uint32_t v_addr = smem_u32(dV);
+      const uint32_t p_addr = smem_u32(sP + (size_t)w * kPBytes);
       if (lane == 0) {
         tc_fence_after();
 #pragma unroll
         for (int kb = 0; kb < kBN / 16; ++kb) {
           const uint64_t ad = sdesc_sw128(p_addr + (uint32_t)kb * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(v_addr + (uint32_t)kb * 2048, kHalf, 1024);
-          mma_bf16_ss(tmem + kColO, ad, bd, idesc_o, (i > 0 || kb > 0) ? 1u : 0u);
+          mma_bf16_ss(tmem + kColO + (uint32_t)w * kD, ad, bd, idesc_o, (i >= 2 || kb > 0) ? 1u : 0u);
         }
-        tc_commit(&bars.kv_empty[st]);
-        tc_commit(&bars.pv_done);
+        tc_commit(&bars.v_empty[st]);
+        tc_commit(&bars.pv_done[w]);
       }
       __syncwarp();
+      if (i + 2 < nt) ok = issue_s(i + 2);   // warpgroup w has read its S tile: it can be reused
     }
     if (!ok) abort_cta(a, b, &s_abort);
-    if (lane == 0) s_consumed = consumed;
+    if (lane == 0) s_k_consumed = k_consumed, s_v_consumed = v_consumed;
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax + epilogue
-    const int q4 = warp - 4;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = (warp - 4) >> 2;
+    const int q4 = warp & 3;                       // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;
     const int r = r0 + row;
     const bool row_ok = r < r_hi;
+    // a warp whose 32 rows are all padding skips the softmax; its P rows are never read into an
+    // output row (each output row depends on its own P row only)
+    const bool warp_live = r0 + q4 * 32 < r_hi;
     const int nl = row / G;
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t s_col = kColS + (uint32_t)wg * kBN, o_col = kColO + (uint32_t)wg * kD;
     const float sl2 = a.scale * kLog2e;
+    uint8_t* sPw = sP + (size_t)wg * kPBytes;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int i = 0; i < nt; ++i) {
-      if (!mbar_wait(&bars.s_full[i & 1], (i >> 1) & 1)) {
+    for (int i = wg; i < nt; i += 2) {
+      const int k = i >> 1;
+      if (!mbar_wait(&bars.s_full[wg], k & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t s0[32], s1[32];
-      tmem_ld32(lane_addr + kColS + (uint32_t)(i & 1) * kBN, s0);
-      tmem_ld32(lane_addr + kColS + (uint32_t)(i & 1) * kBN + 32, s1);
-      tmem_wait_ld();
       const int t = t_begin + i;
       const bool tree = t >= v.nPT;
       const int kbase = tree ? (t - v.nPT) * kBN : t * kBN;
-      const int lim = tree ? v.N : v.L;
-      uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
-      if (tree) {
-        const int wi = kbase >> 5;
-        w0 = sMask[nl * u.W + wi];
-        w1 = (wi + 1 < u.W) ? sMask[nl * u.W + wi + 1] : 0u;
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const bool v0 = row_ok && (kbase + c < lim) && ((w0 >> c) & 1u);
-        const bool v1 = row_ok && (kbase + 32 + c < lim) && ((w1 >> c) & 1u);
-        const float x0 = v0 ? __uint_as_float(s0[c]) * sl2 : -INFINITY;
-        const float x1 = v1 ? __uint_as_float(s1[c]) * sl2 : -INFINITY;
-        s0[c] = __float_as_uint(x0);
-        s1[c] = __float_as_uint(x1);
-        mx = fmaxf(mx, fmaxf(x0, x1));
-      }
       float alpha = 1.f;
       bool resc = false;
-      if (mx != -INFINITY && (m_used == -INFINITY || mx > m_used + kRescaleLog2)) {
-        if (m_used != -INFINITY) {
-          alpha = exp2f(m_used - mx);
-          resc = true;
-        }
-        m_used = mx;
-      }
-      const float mu = m_used == -INFINITY ? 0.f : m_used;
-      float sum = 0.f;
       uint32_t pk[32];
+      if (warp_live) {
+        uint32_t s0[32], s1[32];
+        tmem_ld32(lane_addr + s_col, s0);
+        tmem_ld32(lane_addr + s_col + 32, s1);
+        tmem_wait_ld();
+        float mx;
+        if (!tree && kbase + kBN <= v.L) {
+          // a full prefix tile: every key is visible to every row, no mask work
+          float ma[8];
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const float p0 = exp2f(__uint_as_float(s0[c]) - mu), p1 = exp2f(__uint_as_float(s0[c + 1]) - mu);
-        const float p2 = exp2f(__uint_as_float(s1[c]) - mu), p3 = exp2f(__uint_as_float(s1[c + 1]) - mu);
-        sum += (p0 + p1) + (p2 + p3);
-        pk[c / 2] = pack_bf16x2(p0, p1);
-        pk[16 + c / 2] = pack_bf16x2(p2, p3);
+          for (int q = 0; q < 8; ++q) ma[q] = fmaxf(__uint_as_float(s0[q]), __uint_as_float(s1[q]));
+#pragma unroll
+          for (int c = 8; c < 32; ++c)
+            ma[c & 7] = fmaxf(ma[c & 7], fmaxf(__uint_as_float(s0[c]), __uint_as_float(s1[c])));
+          mx = fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
+          mx = row_ok ? mx * sl2 : -INFINITY;
+        } else {
+          const int lim = tree ? v.N : v.L;
+          uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
+          if (tree) {
+            const int wi = kbase >> 5;
+            w0 = sMask[nl * u.W + wi];
+            w1 = (wi + 1 < u.W) ? sMask[nl * u.W + wi + 1] : 0u;
+          }
+          // fold the key limit into the bit words: bit c survives iff kbase + c < lim
+          const int n0 = lim - kbase;
+          if (n0 < 32) w0 &= n0 <= 0 ? 0u : ((1u << n0) - 1u);
+          if (n0 < 64) w1 &= n0 <= 32 ? 0u : ((1u << (n0 - 32)) - 1u);
+          if (!row_ok) w0 = w1 = 0u;
+          float ma[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) ma[q] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float x0 = ((w0 >> c) & 1u) ? __uint_as_float(s0[c]) : -INFINITY;
+            const float x1 = ((w1 >> c) & 1u) ? __uint_as_float(s1[c]) : -INFINITY;
+            s0[c] = __float_as_uint(x0);
+            s1[c] = __float_as_uint(x1);
+            ma[c & 7] = fmaxf(ma[c & 7], fmaxf(x0, x1));
+          }
+          mx = fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
+          mx = mx * sl2;   // -inf stays -inf (sl2 > 0)
+        }
+        if (mx != -INFINITY && (m_used == -INFINITY || mx > m_used + kRescaleLog2)) {
+          if (m_used != -INFINITY) {
+            alpha = exp2f(m_used - mx);
+            resc = true;
+          }
+          m_used = mx;
+        }
+        const float nmu = m_used == -INFINITY ? 0.f : -m_used;
+        float suma[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          // p = 2^(s * scale * log2(e) - m): one FFMA feeds the exponential (masked s = -inf gives 0)
+          const float p0 = fast_exp2(fmaf(__uint_as_float(s0[c]), sl2, nmu));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(s0[c + 1]), sl2, nmu));
+          const float p2 = fast_exp2(fmaf(__uint_as_float(s1[c]), sl2, nmu));
+          const float p3 = fast_exp2(fmaf(__uint_as_float(s1[c + 1]), sl2, nmu));
+          suma[(c >> 1) & 3] += (p0 + p1) + (p2 + p3);
+          pk[c / 2] = pack_bf16x2(p0, p1);
+          pk[16 + c / 2] = pack_bf16x2(p2, p3);
+        }
+        l = l * alpha + ((suma[0] + suma[1]) + (suma[2] + suma[3]));
       }
-      l = l * alpha + sum;
-      if (i > 0 && !mbar_wait(&bars.pv_done, (i - 1) & 1)) {
+      // this warpgroup's previous P V (tile i - 2) must be done: P buffer free, O up to date
+      if (k >= 1 && !mbar_wait(&bars.pv_done[wg], (k - 1) & 1)) {
         ok = false;
         break;
       }
-      if (__any_sync(0xffffffffu, resc)) {   // warp-collective TMEM read-modify-write of O
+      if (warp_live && __any_sync(0xffffffffu, resc)) {   // warp-collective TMEM read-modify-write of O
         tc_fence_after();
 #pragma unroll
         for (int ch = 0; ch < kD / 32; ++ch) {
           uint32_t o[32];
-          tmem_ld32(lane_addr + kColO + ch * 32, o);
+          tmem_ld32(lane_addr + o_col + ch * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(lane_addr + kColO + ch * 32, o);
+          tmem_st32(lane_addr + o_col + ch * 32, o);
         }
         tmem_wait_st();
       }
-      // P row -> swizzled shared tile (row = TMEM lane), then hand it to the MMA warp
-      uint8_t* prow = sP + (size_t)row * 128;
+      if (warp_live) {   // P row -> swizzled shared tile (row = TMEM lane)
+        uint8_t* prow = sPw + (size_t)row * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full);
+      if (lane == 0) mbar_arrive(&bars.p_full[wg]);
     }
-    if (ok && nt > 0 && !mbar_wait(&bars.pv_done, (nt - 1) & 1)) ok = false;
+    // the warpgroup's last P V product
+    if (ok && nt > wg && !mbar_wait(&bars.pv_done[wg], ((nt - 1 - wg) >> 1) & 1)) ok = false;
     if (!ok) abort_cta(a, b, &s_abort);
-    row_state_m = m_used;
-    row_state_l = l;
+    row_m = m_used;
+    row_l = l;
+    if (wg == 1) s_ml1[row] = make_float2(m_used, l);
   }
+
   // ---------------------------------------------------------------- epilogue / teardown
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (!s_abort) {
-    if (warp >= 4) {
-      const int q4 = warp - 4;
+    if (warp >= 4 && warp < 8) {
+      // merge the two warpgroups' partial results of this row (log-sum-exp), then write it
+      const int q4 = warp & 3;
       const int row = q4 * 32 + lane;
       const int r = r0 + row;
       const bool row_ok = r < r_hi;
       const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-      const float m_used = row_state_m, l = row_state_l;
+      const float2 ml1 = nt > 1 ? s_ml1[row] : make_float2(-INFINITY, 0.f);
+      const float M = fmaxf(row_m, ml1.x);
+      const float Mu = M == -INFINITY ? 0.f : M;
+      const float a0 = exp2f(row_m - Mu);
+      const float a1 = nt > 1 ? exp2f(ml1.x - Mu) : 0.f;
+      const float l = row_l * a0 + ml1.y * a1;
       const bool err = s_err != 0;
       const int i_node = r / G, hh = r % G;
       if (direct) {
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
                               (((size_t)b * a.Nmax + (row_ok ? i_node : 0)) * a.Hq + g * G + hh) * kD;
         const float inv = (l > 0.f && !err) ? 1.f / l : 0.f;
+        const float c0 = a0 * inv, c1 = a1 * inv;
 #pragma unroll
         for (int ch = 0; ch < kD / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + kColO + ch * 32, o);
+          uint32_t o0[32], o1[32];
+          tmem_ld32(lane_addr + kColO + ch * 32, o0);
+          if (nt > 1) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
           tmem_wait_ld();
+          float f[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            f[e] = __uint_as_float(o0[e]) * c0 + (nt > 1 ? __uint_as_float(o1[e]) * c1 : 0.f);
           if (row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              dst[q] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * q]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
-                                  pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv),
-                                  pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv),
-                                  pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv));
-            }
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pack_bf16x2(f[8 * q], f[8 * q + 1]), pack_bf16x2(f[8 * q + 2], f[8 * q + 3]),
+                                  pack_bf16x2(f[8 * q + 4], f[8 * q + 5]), pack_bf16x2(f[8 * q + 6], f[8 * q + 7]));
           }
         }
         if (row_ok && a.lse)
-          a.lse[((size_t)b * a.Nmax + i_node) * a.Hq + g * G + hh] = err ? 0.f : (m_used + __log2f(l)) * kLn2;
+          a.lse[((size_t)b * a.Nmax + i_node) * a.Hq + g * G + hh] = err ? 0.f : (M + __log2f(l)) * kLn2;
       } else {
+        // split-KV partial: unnormalised O relative to M, with (M, l)
         float* wo = reinterpret_cast<float*>(a.workspace);
         const size_t base = (((size_t)b * a.Hkv + g) * u.splits + split) * u.Rmax;
         float* wml = wo + (size_t)a.B * a.Hkv * u.splits * u.Rmax * kD;
 #pragma unroll
         for (int ch = 0; ch < kD / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + kColO + ch * 32, o);
+          uint32_t o0[32], o1[32];
+          tmem_ld32(lane_addr + kColO + ch * 32, o0);
+          if (nt > 1) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
           tmem_wait_ld();
           if (row_ok) {
             float4* dst = reinterpret_cast<float4*>(wo + (base + r) * kD + ch * 32);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
-                                   __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
+            for (int q = 0; q < 8; ++q) {
+              float f[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                f[e] = __uint_as_float(o0[4 * q + e]) * a0 + (nt > 1 ? __uint_as_float(o1[4 * q + e]) * a1 : 0.f);
+              dst[q] = make_float4(f[0], f[1], f[2], f[3]);
+            }
           }
         }
-        if (row_ok) *reinterpret_cast<float2*>(wml + (base + r) * 2) = make_float2(m_used, l);
+        if (row_ok) *reinterpret_cast<float2*>(wml + (base + r) * 2) = make_float2(M, l);
       }
       if (err && split == 0 && mt == 0 && g == 0 && tid == 128) flag_status(a.status, b, TSD_ERR_CAPACITY);
     }
   } else {
     // time-out: let this CTA's own TMA copies and MMAs land (bounded) before freeing TMEM
-    if (tid == 0)
-      for (int i = s_consumed; i < s_issued; ++i) mbar_wait(&bars.kv_full[i % u.stages], (i / u.stages) & 1);
+    if (tid == 0) {
+      for (int i = s_k_consumed; i < s_k_issued; ++i) mbar_wait(&bars.k_full[i % u.ks], (i / u.ks) & 1);
+      for (int i = s_v_consumed; i < s_v_issued; ++i) mbar_wait(&bars.v_full[i % u.vs], (i / u.vs) & 1);
+    }
     if (warp == 1 && lane == 0) {
       tc_commit(&bars.fin);
       mbar_wait(&bars.fin, 0);
@@ -488,13 +568,20 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   u.tps = p.tps, u.splits = p.splits, u.Rmax = p.Rmax, u.mtiles = p.mtiles;
   u.W = (a.Nmax + 31) / 32;
   const uint32_t mask_bytes = (uint32_t)(kBM / G) * u.W * 4;
-  u.stages = 4;
-  auto total = [&](int st) { return 1024 + kQBytes + (uint32_t)st * kStageBytes + kPBytes + mask_bytes; };
-  if (total(u.stages) > 227 * 1024) u.stages = 3;
-  if (total(u.stages) > 227 * 1024) return TSD_ERR_INVALID_ARG;
-  u.p_off = kQBytes + (uint32_t)u.stages * kStageBytes;
-  u.mask_off = u.p_off + kPBytes;
-  const size_t smem = total(u.stages);
+  auto total = [&](int ks, int vs) {
+    return 1024 + kQBytes + (uint32_t)(ks + vs) * kSlot + 2 * kPBytes + mask_bytes;
+  };
+  u.ks = 4, u.vs = 5;
+  const uint32_t limit = 227 * 1024 - 2048;   // leave room for the static shared variables
+  while (total(u.ks, u.vs) > limit && u.vs > 2) {
+    if (u.vs > u.ks) --u.vs; else --u.ks;
+  }
+  if (total(u.ks, u.vs) > limit) return TSD_ERR_INVALID_ARG;
+  u.k_off = kQBytes;
+  u.v_off = u.k_off + (uint32_t)u.ks * kSlot;
+  u.p_off = u.v_off + (uint32_t)u.vs * kSlot;
+  u.mask_off = u.p_off + 2 * kPBytes;
+  const size_t smem = total(u.ks, u.vs);
 
   CUtensorMap mq, mk, mv, mkt, mvt;
   {  // Q [B*Nmax rows][Hq][128] -> box (64, G, 128/G)
@@ -528,8 +615,9 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   }
   cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid(p.mtiles * p.splits, a.Hkv, a.B);
-  attn_umma_kernel<<<grid, kThreadsU, smem, stream>>>(mq, mk, mv, mkt, mvt, a, u);
-  return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+  if (launch_pdl(attn_umma_kernel, grid, dim3(kThreadsU), smem, stream, mq, mk, mv, mkt, mvt, a, u) != cudaSuccess)
+    return TSD_ERR_CUDA;
+  return TSD_OK;
 }
 
 }  // namespace tsd

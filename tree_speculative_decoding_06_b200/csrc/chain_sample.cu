@@ -72,6 +72,7 @@ __device__ __forceinline__ void merge(float& zm, double& s, float zm2, double s2
 template <typename T>
 __global__ void __launch_bounds__(kThreads) stats_kernel(const T* __restrict__ zp, const T* __restrict__ zq, int V,
                                                          int K, Temp tc, int chunks, Stat* __restrict__ part) {
+  pdl_trigger();   // the scan reads inputs only; pdl_wait() comes before the partial is written
   const int c = blockIdx.x, r = blockIdx.y, b = blockIdx.z;
   const T* row = chain_row(zp, zq, K, V, b, r);
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
@@ -116,6 +117,7 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(const T* __restrict__ z
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) szm[warp] = zm, ss[warp] = s;
   __syncthreads();
+  pdl_wait();
   if (threadIdx.x == 0) {
     float M = -INFINITY;
     double S = 0.0;
@@ -142,7 +144,8 @@ template <typename T>
 __device__ int decide_warp(const T* zp, const T* zq, const int32_t* x, const float* u, const Stat* part, int chunks,
                            int V, int K, const Temp& tc, int b, Stat* st, float* ex) {
   const int lane = threadIdx.x & 31;
-  for (int r = lane; r < 2 * K + 1; r += 32) st[r] = merge_stats(part + ((size_t)b * (2 * K + 1) + r) * chunks, chunks, tc.c);
+  for (int r = lane; r < 2 * K + 1; r += 32)
+    st[r] = merge_stats(part + ((size_t)b * (2 * K + 1) + r) * chunks, chunks, tc.c);
   __syncwarp();
   for (int k = lane; k < K; k += 32) {
     const int xk = x[(size_t)b * K + k];
@@ -199,6 +202,8 @@ __global__ void __launch_bounds__(kThreads) mass_kernel(const T* __restrict__ zp
                                                         int V, int K, Temp tc, int chunks,
                                                         const Stat* __restrict__ part, double* __restrict__ mass,
                                                         int* __restrict__ jout) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ Stat s_st[];     // 2K+1 statistics, then 2K floats of draft exponentials
   __shared__ int s_j;
   const int c = blockIdx.x, b = blockIdx.y;
@@ -279,6 +284,8 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
                                                           const int* __restrict__ jin,
                                                           int32_t* __restrict__ accept_len,
                                                           int32_t* __restrict__ out_tokens) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ Final s_f;
   __shared__ int s_c;
   __shared__ double s_thr;
@@ -369,17 +376,19 @@ tsd_status launch_chain_sample_stochastic(const void* zp, const void* zq, tsd_dt
   if (dtype == TSD_BF16) {
     auto p = reinterpret_cast<const __nv_bfloat16*>(zp);
     auto q = reinterpret_cast<const __nv_bfloat16*>(zq);
-    stats_kernel<__nv_bfloat16><<<g1, kThreads, 0, stream>>>(p, q, V, K, tc, chunks, part);
-    mass_kernel<__nv_bfloat16><<<g2, kThreads, st_smem, stream>>>(p, q, x, u, V, K, tc, chunks, part, mass, jbuf);
-    select_kernel<__nv_bfloat16><<<B, kThreads, 0, stream>>>(p, q, x, u, V, K, tc, chunks, part, mass, jbuf,
-                                                             accept_len, out_tokens);
+    launch_pdl(stats_kernel<__nv_bfloat16>, g1, dim3(kThreads), 0, stream, p, q, V, K, tc, chunks, part);
+    launch_pdl(mass_kernel<__nv_bfloat16>, g2, dim3(kThreads), st_smem, stream, p, q, x, u, V, K, tc, chunks,
+               (const Stat*)part, mass, jbuf);
+    launch_pdl(select_kernel<__nv_bfloat16>, dim3(B), dim3(kThreads), 0, stream, p, q, x, u, V, K, tc, chunks,
+               (const Stat*)part, (const double*)mass, (const int*)jbuf, accept_len, out_tokens);
   } else {
     auto p = reinterpret_cast<const float*>(zp);
     auto q = reinterpret_cast<const float*>(zq);
-    stats_kernel<float><<<g1, kThreads, 0, stream>>>(p, q, V, K, tc, chunks, part);
-    mass_kernel<float><<<g2, kThreads, st_smem, stream>>>(p, q, x, u, V, K, tc, chunks, part, mass, jbuf);
-    select_kernel<float><<<B, kThreads, 0, stream>>>(p, q, x, u, V, K, tc, chunks, part, mass, jbuf, accept_len,
-                                                     out_tokens);
+    launch_pdl(stats_kernel<float>, g1, dim3(kThreads), 0, stream, p, q, V, K, tc, chunks, part);
+    launch_pdl(mass_kernel<float>, g2, dim3(kThreads), st_smem, stream, p, q, x, u, V, K, tc, chunks,
+               (const Stat*)part, mass, jbuf);
+    launch_pdl(select_kernel<float>, dim3(B), dim3(kThreads), 0, stream, p, q, x, u, V, K, tc, chunks, (const Stat*)part,
+               (const double*)mass, (const int*)jbuf, accept_len, out_tokens);
   }
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }

@@ -9,6 +9,15 @@
 
 namespace tsd {
 
+// Programmatic dependent launch.  Every kernel of the library is launched with programmatic
+// stream serialisation: it may be scheduled while the previous kernel in the stream is still
+// running.  pdl_trigger() lets the next kernel be scheduled; pdl_wait() blocks until the previous
+// kernel has completed and its writes are visible.  Every kernel calls pdl_wait() on every path
+// before it writes anything an earlier kernel may read, and before it reads anything an earlier
+// kernel writes, so "previous kernel complete" stays transitive down the stream.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 // Record a device-detected error for sequence b unless an earlier one is already there.
 __device__ __forceinline__ void flag_status(int32_t* status, int b, int code, int detail = 0) {
   atomicCAS(status + b, 0, code | (detail << 8));

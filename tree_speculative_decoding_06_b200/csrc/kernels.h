@@ -6,9 +6,28 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "tsd.h"
 
 namespace tsd {
+
+// Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger in common.cuh).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Split-KV plan of one attention launch: a CTA covers BM query rows of one (sequence, KV head)
 // and `tps` key tiles of BN keys; the keys of sequence b are its prefix tiles followed by its

@@ -34,6 +34,8 @@ __device__ __forceinline__ size_t row_off(const CommitArgs& a, int b, int h, int
 }
 
 __global__ void __launch_bounds__(kThreads) kv_commit_kernel(const CommitArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(16) uint8_t s_stage[];
   __shared__ int s_src[257];
   __shared__ int s_bad;
@@ -135,8 +137,7 @@ tsd_status launch_kv_commit(const CommitArgs& a, cudaStream_t stream) {
     if (smem > 200 * 1024) return TSD_ERR_INVALID_ARG;   // one row of every head must fit on chip
     if (smem > 48 * 1024) cudaFuncSetAttribute(kv_commit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   }
-  kv_commit_kernel<<<a.B, kThreads, smem, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+  return launch_pdl(kv_commit_kernel, dim3(a.B), dim3(kThreads), smem, stream, a) == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }
 
 }  // namespace tsd

@@ -17,6 +17,8 @@ __global__ void tree_prepare_kernel(const int32_t* __restrict__ parent, const in
                                     int Nmax, int Dmax, int forest, int32_t* __restrict__ parent_s,
                                     int32_t* __restrict__ depth_s, int32_t* __restrict__ anc,
                                     uint32_t* __restrict__ anc_bits, int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x;
   const int N = num_nodes ? num_nodes[b] : Nmax;
   const int32_t* par = parent + (size_t)b * Nmax;
@@ -98,8 +100,9 @@ tsd_status launch_tree_prepare(const int32_t* parent, const int32_t* num_nodes, 
                                int32_t* status, cudaStream_t stream) {
   if (B == 0) return TSD_OK;
   const int threads = Nmax + 1 >= 256 ? 256 : ((Nmax + 1 + 31) / 32) * 32;
-  tree_prepare_kernel<<<B, threads, 0, stream>>>(parent, num_nodes, Nmax, Dmax, forest, parent_s, depth, anc,
-                                                 anc_bits, status);
+  if (launch_pdl(tree_prepare_kernel, dim3(B), dim3(threads), 0, stream, parent, num_nodes, Nmax, Dmax, forest, parent_s,
+                 depth, anc, anc_bits, status) != cudaSuccess)
+    return TSD_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }
 
