@@ -64,6 +64,30 @@ def tokens_per_step(inp) -> int:
     return int(np.asarray(inp["num_nodes"]).sum())
 
 
+def rank_workload(name: str, rank: int, batch: int = 0):
+    """The workload one rank verifies: the named shape with its own seed (weak scaling: every rank
+    owns a full batch of its own sequences; no data moves between ranks)."""
+    w = W.WORKLOADS[name]
+    if batch:
+        w = w.scaled(B=batch)
+    return w, w.seed + 1000 * rank
+
+
+def reduce_over_ranks(values, world: int, device=None):
+    """Max over ranks of per-rank device times (ms): the slowest rank bounds the step."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def aggregate_rate(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the tokens every rank verified over the max-over-ranks time."""
+    return world * tokens_per_rank_step * steps / (max_ms * 1e-3)
+
+
 def read_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -160,10 +184,8 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = W.WORKLOADS[args.workload]
-    if args.batch:
-        w = w.scaled(B=args.batch)
-    inp = W.make_inputs(w, seed=w.seed + 1000 * rank, nan_guard=False)
+    w, seed = rank_workload(args.workload, rank, args.batch)
+    inp = W.make_inputs(w, seed=seed, nan_guard=False)
     tok = tokens_per_step(inp)
     x0 = to_device(inp, dev)
     per_set = sum(v.numel() * v.element_size() for v in x0.values() if isinstance(v, torch.Tensor))
@@ -234,10 +256,7 @@ def run_ours(args, rank, world, local_rank):
         wall = time.perf_counter() - t_wall
     if world > 1:
         dist.barrier()
-    t = torch.tensor([step_ms, attn_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, attn_ms = float(t[0]), float(t[1])
+    step_ms, attn_ms = reduce_over_ranks([step_ms, attn_ms], world, dev)
 
     # status check: every sequence of every set must be clean
     bad = sum(int((st.status != 0).sum()) for st in steps)
@@ -273,10 +292,7 @@ def run_ours(args, rank, world, local_rank):
                 host_out[k].copy_(getattr(steps[0], k), non_blocking=True)
         e1.record(stream)
     torch.cuda.synchronize(dev)
-    e_ms = torch.tensor([e0.elapsed_time(e1) / e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-    e_ms = float(e_ms[0])
+    e_ms = reduce_over_ranks([e0.elapsed_time(e1) / e_steps], world, dev)[0]
 
     # launches of our kernels per step: prepare, attention (+ merge), acceptance, commit
     attn_ws = steps[0].attn_ws.numel() > 1
@@ -290,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
         alg = attn_algorithmic_bytes(inp)
         achieved = alg / (attn_ms * 1e-3) / 1e9
         traffic = recorded_traffic(args.workload)
-        value = world * tok * args.steps / (step_ms * 1e-3)
+        value = aggregate_rate(tok, world, args.steps, step_ms)
         res = {
             "metric": "verified tree tokens/s (whole verify step: prepare + tree attention + acceptance + commit)",
             "value": round(value, 1),
@@ -316,7 +332,7 @@ def run_ours(args, rank, world, local_rank):
                          "kernel": "tsd_tree_verify_attn (split kernel + merge)",
                          "algorithmic_bytes_per_launch": alg, "attn_us_per_launch": round(attn_ms * 1e3, 3),
                          "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"},
-            "e2e": {"value": round(world * tok / (e_ms * 1e-3), 1), "unit": "tokens/s",
+            "e2e": {"value": round(aggregate_rate(tok, world, 1, e_ms), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e_ms, 4)},
             "gpu_launches": launches,

@@ -524,14 +524,28 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
   p.max_tiles = (Lcap + p.BN - 1) / p.BN + (Nmax + p.BN - 1) / p.BN;
   const long long base = (long long)B * Hkv * p.mtiles;
   const int sms = device_sm_count();
-  const int want = base >= 2LL * sms ? 1 : (int)((2LL * sms + base - 1) / (base > 0 ? base : 1));
-  const int min_tps = (3 * p.BM / 2 + p.BN - 1) / p.BN;
-  int tps = (p.max_tiles + want - 1) / want;
-  if (tps < min_tps) tps = min_tps;
-  if (tps < 1) tps = 1;
-  if (tps > p.max_tiles) tps = p.max_tiles > 0 ? p.max_tiles : 1;
-  p.tps = tps;
-  p.splits = (p.max_tiles + tps - 1) / tps;
+  // Split count: the CTAs of one launch run in waves of one CTA per SM, a CTA costs its tiles plus a
+  // fixed overhead (set-up, pipeline fill, epilogue) of about two tiles, and every split adds
+  // partials to write and merge.
+  // Minimise waves * (tiles per split + overhead) over the split counts that keep a split at least
+  // min_tps tiles long (partials must stay small next to the K/V they summarise).
+  const int min_tps = dtype == TSD_BF16 ? 2 : (3 * p.BM / 2 + p.BN - 1) / p.BN;
+  const double overhead = 2.0;
+  int best_tps = p.max_tiles > 0 ? p.max_tiles : 1;
+  double best_cost = 1e300;
+  for (int s = 1; s <= 64; ++s) {
+    int tps = (p.max_tiles + s - 1) / s;
+    if (tps < 1) tps = 1;
+    if (s > 1 && tps < min_tps) break;
+    const int splits = (p.max_tiles + tps - 1) / tps;
+    const long long ctas = base * splits;
+    const double waves = (double)((ctas + sms - 1) / sms);
+    // each extra split adds a partial row set to write and merge
+    const double cost = waves * (tps + overhead) + (splits > 1 ? 0.35 * splits : 0.0);
+    if (cost < best_cost - 1e-9) best_cost = cost, best_tps = tps;
+  }
+  p.tps = best_tps;
+  p.splits = (p.max_tiles + p.tps - 1) / p.tps;
   if (p.splits < 1) p.splits = 1;
   p.ws_bytes = p.splits > 1 ? (size_t)B * Hkv * p.splits * p.Rmax * (d + 2) * sizeof(float) : 0;
   return p;

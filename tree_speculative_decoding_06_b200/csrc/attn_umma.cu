@@ -10,8 +10,9 @@
 //     box by block, the tree's K/V by node for one KV head) into separate rings: a K slot is
 //     released as soon as S = Q K^T has read it, a V slot after P V, so loads run several tiles
 //     ahead of the math;
-//   * one thread issues tcgen05.mma: S into one of two TMEM tiles (128 lanes x 64 fp32 columns)
-//     and O += P V into one of two 128 x 128 fp32 TMEM accumulators;
+//   * one thread (warp 3) issues tcgen05.mma: S into one of two TMEM tiles (128 lanes x 64 fp32
+//     columns) and O += P V into one of two 128 x 128 fp32 TMEM accumulators, with descriptors
+//     built once and advanced by constants;
 //   * two softmax warpgroups take alternate tiles (even / odd), each with its own S tile, P
 //     buffer, O accumulator and running (max, sum) -- a split of the key range inside the CTA,
 //     merged by log-sum-exp in the epilogue.  In a warpgroup each warp owns one TMEM lane
@@ -84,10 +85,28 @@ __device__ __forceinline__ void abort_cta(const AttnArgs& a, int b, volatile int
   }
 }
 
+// Block ids of the boxes of prefix tile t (paged caches): loaded one tile ahead by the producers so
+// the table reads never wait in line behind the TMA issues.
+struct TileBlocks {
+  int blk[8];
+};
+__device__ __forceinline__ void fetch_blocks(const AttnArgs& a, const SeqView& v, const UParams& u, int b, int t,
+                                             TileBlocks& tb) {
+  if (a.block_table == nullptr || t >= v.nPT) return;
+  const int pos0 = t * kBN;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int seg = k * u.box_rows;
+    if (seg < kBN) tb.blk[k] = a.block_table[(size_t)b * a.max_blocks + min((pos0 + seg) >> a.block_shift,
+                                                                             a.max_blocks - 1)];
+  }
+}
+
 // TMA loads of one 64-key tile (K or V half pair) of sequence b, KV head g into `dst`.
 __device__ __forceinline__ void load_tile(const AttnArgs& a, const SeqView& v, const UParams& u, int b, int g,
                                           int t, uint8_t* dst, const CUtensorMap* cache_map,
-                                          const CUtensorMap* tree_map, uint64_t* bar, int* s_err) {
+                                          const CUtensorMap* tree_map, uint64_t* bar, int* s_err,
+                                          const TileBlocks& tb) {
   if (t < v.nPT) {
     const int pos0 = t * kBN;
     if (a.block_table == nullptr) {
@@ -96,10 +115,12 @@ __device__ __forceinline__ void load_tile(const AttnArgs& a, const SeqView& v, c
       tma_load_2d(dst + kHalf, cache_map, 64, y, bar);
     } else {
       const int bs_mask = (1 << a.block_shift) - 1;
-      for (int seg = 0; seg < kBN; seg += u.box_rows) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int seg = k * u.box_rows;
+        if (seg >= kBN) break;
         const int pos = pos0 + seg;
-        const int bi = min(pos >> a.block_shift, a.max_blocks - 1);
-        int blk = a.block_table[(size_t)b * a.max_blocks + bi];
+        int blk = tb.blk[k];
         if (blk < 0 || blk >= a.num_blocks) {
           if (pos < v.L) *s_err = 1;
           blk = 0;
@@ -175,11 +196,11 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     fence_barrier_init();
     fence_proxy_async();
   }
-  if (warp == 1) {
+  if (warp == 3) {
     tmem_alloc(&s_tmem, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 3) {
+  if (warp == 1) {
     if (t_begin + nt > v.nPT) build_mask(a, b, node0, nodes_per_tile, u.W, sMask, v.N, lane, 32);
   }
   tc_fence_before();
@@ -196,14 +217,18 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       tma_load_3d(sQ, &tmQ, 0, g * G, zq, &bars.q_full);
       tma_load_3d(sQ + kQBytes / 2, &tmQ, 64, g * G, zq, &bars.q_full);
       int issued = 0;
+      TileBlocks nxt;
+      fetch_blocks(a, v, u, b, t_begin, nxt);
       for (int i = 0; i < nt && !s_abort; ++i) {
+        const TileBlocks cur = nxt;
+        if (i + 1 < nt) fetch_blocks(a, v, u, b, t_begin + i + 1, nxt);
         const int st = i % u.ks;
         if (i >= u.ks && !mbar_wait(&bars.k_empty[st], ((i / u.ks) - 1) & 1)) {
           abort_cta(a, b, &s_abort);
           break;
         }
         mbar_expect_tx(&bars.k_full[st], kSlot);
-        load_tile(a, v, u, b, g, t_begin + i, sK + (size_t)st * kSlot, &tmK, &tmKt, &bars.k_full[st], &s_err);
+        load_tile(a, v, u, b, g, t_begin + i, sK + (size_t)st * kSlot, &tmK, &tmKt, &bars.k_full[st], &s_err, cur);
         ++issued;
       }
       s_k_issued = issued;
@@ -212,23 +237,32 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     // ------------------------------------------------------------ V producer (one thread)
     if (lane == 0) {
       int issued = 0;
+      TileBlocks nxt;
+      fetch_blocks(a, v, u, b, t_begin, nxt);
       for (int i = 0; i < nt && !s_abort; ++i) {
+        const TileBlocks cur = nxt;
+        if (i + 1 < nt) fetch_blocks(a, v, u, b, t_begin + i + 1, nxt);
         const int st = i % u.vs;
         if (i >= u.vs && !mbar_wait(&bars.v_empty[st], ((i / u.vs) - 1) & 1)) {
           abort_cta(a, b, &s_abort);
           break;
         }
         mbar_expect_tx(&bars.v_full[st], kSlot);
-        load_tile(a, v, u, b, g, t_begin + i, sV + (size_t)st * kSlot, &tmV, &tmVt, &bars.v_full[st], &s_err);
+        load_tile(a, v, u, b, g, t_begin + i, sV + (size_t)st * kSlot, &tmV, &tmVt, &bars.v_full[st], &s_err, cur);
         ++issued;
       }
       s_v_issued = issued;
     }
-  } else if (warp == 1) {
+  } else if (warp == 3) {
     // ------------------------------------------------------------ MMA issuer (one thread)
+    // Warp 3 shares its SM sub-partition with row quarter 3, which is padding in small-row tiles.
+    // Descriptors are built once; a k-step advances the 14-bit start-address field by a constant.
     const uint32_t idesc_s = idesc_bf16(kBM, kBN, false);
     const uint32_t idesc_o = idesc_bf16(kBM, kD, true);
-    const uint32_t q_addr = smem_u32(sQ);
+    const uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dk = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dv = sdesc_sw128(smem_u32(sV), kHalf, 1024);
+    const uint64_t dp = sdesc_sw128(smem_u32(sP), 16, 1024);
     bool ok = mbar_wait(&bars.q_full, 0);
     int k_consumed = 0, v_consumed = 0;
     // S(j) = Q K(j)^T into warpgroup (j & 1)'s S tile; frees the K slot when done
@@ -236,16 +270,15 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       const int st = j % u.ks;
       if (!mbar_wait(&bars.k_full[st], (j / u.ks) & 1)) return false;
       ++k_consumed;
-      const uint32_t k_addr = smem_u32(sK + (size_t)st * kSlot);
-      const uint32_t d = tmem + kColS + (uint32_t)(j & 1) * kBN;
       if (lane == 0) {
         tc_fence_after();
+        const uint64_t bk = dk + (uint64_t)((st * kSlot) >> 4);
+        const uint32_t d = tmem + kColS + (uint32_t)(j & 1) * kBN;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t half = (uint32_t)(kk >> 2), within = (uint32_t)(kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(q_addr + half * (kQBytes / 2) + within, 16, 1024);
-          const uint64_t bd = sdesc_sw128(k_addr + half * kHalf + within, 16, 1024);
-          mma_bf16_ss(d, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t off_q = ((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4;
+          const uint32_t off_k = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(d, dq + off_q, bk + off_k, idesc_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bars.k_empty[st]);
         tc_commit(&bars.s_full[j & 1]);
@@ -270,8 +303,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       // zero V rows past the valid keys of a partial tile (its TMA box may hold stale rows)
       const int t = t_begin + i;
       const int nv = t < v.nPT ? min(kBN, v.L - t * kBN) : min(kBN, v.N - (t - v.nPT) * kBN);
-      uint8_t* dV = sV + (size_t)st * kSlot;
       if (nv < kBN) {
+        uint8_t* dV = sV + (size_t)st * kSlot;
         const int nchunks = (kBN - nv) * 8;   // 16-byte chunks per half
         for (int c = lane; c < 2 * nchunks; c += 32) {
           const int half = c / nchunks, cc = c % nchunks;
@@ -280,16 +313,14 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         fence_proxy_async();
       }
       __syncwarp();
-      const uint32_t v_addr = smem_u32(dV);
-      const uint32_t p_addr = smem_u32(sP + (size_t)w * kPBytes);
       if (lane == 0) {
         tc_fence_after();
+        const uint64_t bv = dv + (uint64_t)((st * kSlot) >> 4);
+        const uint64_t ap = dp + (uint64_t)((w * kPBytes) >> 4);
+        const uint32_t d = tmem + kColO + (uint32_t)w * kD;
 #pragma unroll
-        for (int kb = 0; kb < kBN / 16; ++kb) {
-          const uint64_t ad = sdesc_sw128(p_addr + (uint32_t)kb * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(v_addr + (uint32_t)kb * 2048, kHalf, 1024);
-          mma_bf16_ss(tmem + kColO + (uint32_t)w * kD, ad, bd, idesc_o, (i >= 2 || kb > 0) ? 1u : 0u);
-        }
+        for (int kb = 0; kb < kBN / 16; ++kb)
+          mma_bf16_ss(d, ap + (uint32_t)(kb * 2), bv + (uint32_t)(kb * 128), idesc_o, (i >= 2 || kb > 0) ? 1u : 0u);
         tc_commit(&bars.v_empty[st]);
         tc_commit(&bars.pv_done[w]);
       }
@@ -509,14 +540,14 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       for (int i = s_k_consumed; i < s_k_issued; ++i) mbar_wait(&bars.k_full[i % u.ks], (i / u.ks) & 1);
       for (int i = s_v_consumed; i < s_v_issued; ++i) mbar_wait(&bars.v_full[i % u.vs], (i / u.vs) & 1);
     }
-    if (warp == 1 && lane == 0) {
+    if (warp == 3 && lane == 0) {
       tc_commit(&bars.fin);
       mbar_wait(&bars.fin, 0);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 3) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -571,10 +602,10 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   auto total = [&](int ks, int vs) {
     return 1024 + kQBytes + (uint32_t)(ks + vs) * kSlot + 2 * kPBytes + mask_bytes;
   };
-  u.ks = 4, u.vs = 5;
+  u.ks = 5, u.vs = 4;   // K is consumed first (by S = Q K^T), so its ring runs further ahead
   const uint32_t limit = 227 * 1024 - 2048;   // leave room for the static shared variables
   while (total(u.ks, u.vs) > limit && u.vs > 2) {
-    if (u.vs > u.ks) --u.vs; else --u.ks;
+    if (u.ks > u.vs) --u.ks; else --u.vs;
   }
   if (total(u.ks, u.vs) > limit) return TSD_ERR_INVALID_ARG;
   u.k_off = kQBytes;
