@@ -99,7 +99,7 @@ def read_peaks():
 
 def attn_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("attn.cu", "common.cuh", "kernels.h"):
+    for f in ("attn.cu", "attn_umma.cu", "attn_common.cuh", "umma.cuh", "common.cuh", "kernels.h"):
         with open(os.path.join(ROOT, "tree_speculative_decoding_06_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -294,11 +294,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     e_ms = reduce_over_ranks([e0.elapsed_time(e1) / e_steps], world, dev)[0]
 
-    # launches of our kernels per step: prepare, attention (+ merge), acceptance, commit
-    attn_ws = steps[0].attn_ws.numel() > 1
-    acc_k = 2 if steps[0].accept == "greedy" else (3 if float(inp.get("T", 1.0)) > 0 else 2)
-    per_step = 1 + 1 + int(attn_ws) + acc_k + 1
-    launches = per_step * args.steps + (1 + int(attn_ws)) * n_attn
+    # launches of our kernels: per step (prepare, attention (+ merge), fused acceptance + commit,
+    # or the chain sampler and the commit), plus the attention-only graph
+    per_step = steps[0].launches_per_step()
+    launches = per_step * args.steps + (1 + int(steps[0].splits_merge)) * n_attn
 
     res = None
     if rank == 0:

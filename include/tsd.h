@@ -286,6 +286,47 @@ tsd_status tsd_kv_commit_paged(void *k_pages, void *v_pages, int num_blocks, int
                                int d, int Dmax, tsd_dtype dtype, tsd_commit_mode mode, int32_t *status,
                                void *stream);
 
+/* ---------------------------------------------------------------------------------------
+ * tsd_tree_accept_commit -- greedy tree acceptance and the commit of the accepted path in one
+ * step, with an optional splice of the emitted tokens into a device token history
+ * ([EP] sec. 2: commit follows the accepted path's indices; [SO] "EAGLE": longest matching
+ * branch plus the target's own token; the accepted length drives the next step's cache length
+ * on the device, with no host synchronisation).
+ *
+ * Same results as tsd_tree_accept_greedy followed by tsd_kv_commit[_paged] with the same
+ * arguments: accept_len, path and out_tokens as there, the cache rows and prefix_len as there.
+ * In addition, when history is not NULL, for every committed sequence
+ *   history[b, H .. H+A] <- out_tokens[b, 0 .. A],  history_len[b] = H + A + 1,
+ * with H = history_len[b]; H < 0 or H + A + 1 > history_cap flags TSD_ERR_CAPACITY before any
+ * cache write (the acceptance outputs are still written).
+ *
+ *   cache       the committed K/V cache (struct below: contiguous when block_table is NULL,
+ *               else paged with the layout of tsd_tree_verify_attn_paged); prefix_len in/out
+ *   mode        TSD_COMMIT_PATH or TSD_COMMIT_INPLACE (LENGTH commits the first A+1 tree rows)
+ *   history     [B, history_cap] int32 device memory, or NULL (no splice; history_len unused)
+ *   workspace   >= tsd_tree_accept_greedy_workspace_size(B, Nmax, V) bytes
+ * Errors as the two calls it replaces.  Two kernel launches on `stream` (the vocabulary scan,
+ * then one CTA per sequence for acceptance, commit and splice); nothing is allocated.
+ * --------------------------------------------------------------------------------------- */
+typedef struct tsd_kv_cache {
+  void *k;                     /* [B, Hkv, Lmax, d] or [num_blocks, Hkv, block_size, d] */
+  void *v;
+  int32_t *prefix_len;         /* [B] committed lengths, advanced on the device */
+  int Lmax;                    /* contiguous capacity per sequence (ignored when paged) */
+  const int32_t *block_table;  /* [B, max_blocks] block ids, or NULL for the contiguous layout */
+  int max_blocks;
+  int block_size;              /* power of two in [8, 256] when paged */
+  int num_blocks;
+} tsd_kv_cache;
+
+tsd_status tsd_tree_accept_commit(const void *logits, tsd_dtype logits_dtype, int V, const int32_t *tokens,
+                                  const int32_t *parent_s, const int32_t *num_nodes, const int32_t *root_key,
+                                  int B, int Nmax, int Dmax, const tsd_kv_cache *cache, const void *k_tree,
+                                  const void *v_tree, int Hkv, int d, tsd_dtype kv_dtype, tsd_commit_mode mode,
+                                  int32_t *history, int history_cap, int32_t *history_len, int32_t *accept_len,
+                                  int32_t *path, int32_t *out_tokens, void *workspace, size_t ws_bytes,
+                                  int32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,6 +52,16 @@ _SIGS = {
 }
 
 
+class KVCacheDesc(C.Structure):
+    """tsd_kv_cache: the committed cache as the fused acceptance + commit call sees it."""
+    _fields_ = [("k", _P), ("v", _P), ("prefix_len", _P), ("Lmax", _I), ("block_table", _P), ("max_blocks", _I),
+                ("block_size", _I), ("num_blocks", _I)]
+
+
+_SIGS["tsd_tree_accept_commit"] = (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, C.POINTER(KVCacheDesc), _P, _P, _I,
+                                        _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P, _P])
+
+
 class TsdError(RuntimeError):
     pass
 
@@ -298,6 +308,41 @@ def kv_commit_paged(k_pages, v_pages, block_table, prefix_len, k_tree, v_tree, p
                                    _stream(stream))
     _check(rc, "tsd_kv_commit_paged")
     return status
+
+
+def tree_accept_commit(logits, tokens, parent_s, k_cache, v_cache, prefix_len, k_tree, v_tree, num_nodes=None,
+                       root_key=None, Dmax: int = 8, mode: str = "path", block_table=None, history=None,
+                       history_len=None, accept_len=None, path=None, out_tokens=None, workspace=None, status=None,
+                       stream=None):
+    """Greedy acceptance fused with the commit of the accepted path (tsd_tree_accept_commit).
+    k_cache/v_cache are [B,Hkv,Lmax,d], or pages [num_blocks,Hkv,block,d] when block_table is
+    given.  With history [B,cap] and history_len [B] the emitted tokens are appended on the
+    device.  Returns the acceptance outputs; the cache, prefix_len and history change in place."""
+    B, Nmax, V = logits.shape
+    accept_len = _empty((B,), torch.int32, logits) if accept_len is None else accept_len
+    path = _empty((B, Dmax + 1), torch.int32, logits) if path is None else path
+    out_tokens = _empty((B, Dmax + 1), torch.int32, logits) if out_tokens is None else out_tokens
+    if status is None:
+        status = torch.zeros(B, dtype=torch.int32, device=logits.device)
+    nbytes = tree_accept_greedy_workspace_size(B, Nmax, V)
+    workspace = _ws(nbytes, logits, workspace)
+    if block_table is not None:
+        nblk, Hkv, bs, d = k_cache.shape
+        desc = KVCacheDesc(_ptr(k_cache), _ptr(v_cache), _i32(prefix_len, "prefix_len"), 0,
+                           _i32(block_table, "block_table"), block_table.shape[1], bs, nblk)
+    else:
+        _, Hkv, Lmax, d = k_cache.shape
+        desc = KVCacheDesc(_ptr(k_cache), _ptr(v_cache), _i32(prefix_len, "prefix_len"), Lmax, None, 0, 0, 0)
+    cap = history.shape[1] if history is not None else 0
+    rc = lib().tsd_tree_accept_commit(_ptr(logits), _dt(logits), V, _i32(tokens, "tokens"),
+                                      _i32(parent_s, "parent_s"), _i32(num_nodes, "num_nodes"),
+                                      _i32(root_key, "root_key"), B, Nmax, Dmax, C.byref(desc), _ptr(k_tree),
+                                      _ptr(v_tree), Hkv, d, _dt(k_cache), COMMIT_MODES[mode],
+                                      _i32(history, "history"), cap, _i32(history_len, "history_len"),
+                                      _ptr(accept_len), _ptr(path), _ptr(out_tokens), _ptr(workspace), nbytes,
+                                      _ptr(status), _stream(stream))
+    _check(rc, "tsd_tree_accept_commit")
+    return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
 
 
 from .step import VerifyStep  # noqa: E402,F401

@@ -14,6 +14,7 @@
 #include <climits>
 #include <mutex>
 
+#include "accept_body.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -92,17 +93,6 @@ __global__ void __launch_bounds__(kThreads) row_argmax_chunks(const T* __restric
   }
 }
 
-__device__ __forceinline__ int merge_argmax(const float2* p, int chunks) {
-  float bv = -INFINITY;
-  int bi = INT_MAX;
-  for (int c = 0; c < chunks; ++c) {
-    const float v = p[c].x;
-    const int i = __float_as_int(p[c].y);
-    if (better(v, i, bv, bi)) bv = v, bi = i;
-  }
-  return bi == INT_MAX ? 0 : bi;
-}
-
 // Per-tree acceptance: t*(node), accepted set by walking each node's ancestors, deepest node.
 __global__ void __launch_bounds__(kThreads) tree_accept_kernel(const float2* __restrict__ part, int chunks,
                                                                const int32_t* __restrict__ tokens,
@@ -112,67 +102,14 @@ __global__ void __launch_bounds__(kThreads) tree_accept_kernel(const float2* __r
                                                                int Dmax, int32_t* __restrict__ accept_len,
                                                                int32_t* __restrict__ path,
                                                                int32_t* __restrict__ out_tokens,
-                                                               const int32_t* __restrict__ status) {
+                                                               const int32_t* __restrict__ status, int staged) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ int32_t s_tstar[];
-  __shared__ int s_hit, s_best;
-  const int b = blockIdx.x;
-  const int N = num_nodes ? num_nodes[b] : Nmax;
-  const int32_t* tok = tokens + (size_t)b * Nmax;
-  const int32_t* ps = parent_s + (size_t)b * (Nmax + 1);
-  int32_t* prow = path + (size_t)b * (Dmax + 1);
-  int32_t* orow = out_tokens + (size_t)b * (Dmax + 1);
-  const bool live = status[b] == 0 && N > 0 && N <= Nmax;
-  if (threadIdx.x == 0) s_hit = INT_MAX, s_best = -1;
-  for (int i = threadIdx.x; live && i < N; i += blockDim.x)
-    s_tstar[i] = merge_argmax(part + ((size_t)b * Nmax + i) * chunks, chunks);
-  __syncthreads();
-  if (live && root_key) {
-    const int key = root_key[b];
-    for (int i = threadIdx.x; i < N; i += blockDim.x)
-      if (ps[i + 1] == 0 && tok[i] == key) atomicMin(&s_hit, i);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; live && i < N; i += blockDim.x) {
-    // accepted iff every edge on the root->i path matches and the root is accepted
-    bool ok = true;
-    int s = i + 1, d = 0;
-    for (;;) {
-      const int p = ps[s];
-      if (p == 0) {
-        if (root_key) ok = ok && (s - 1 == s_hit);
-        break;
-      }
-      if (p >= s || d >= Dmax) {   // prepare guarantees neither; stay bounded anyway
-        ok = false;
-        break;
-      }
-      ok = ok && (tok[s - 1] == s_tstar[p - 1]);
-      s = p;
-      ++d;
-      if (!ok) break;
-    }
-    if (ok) atomicMax(&s_best, (d << 20) | (0xFFFFF - i));
-  }
-  __syncthreads();
-  if (threadIdx.x != 0) return;
-  const int best = live ? s_best : -1;
-  if (best < 0) {
-    accept_len[b] = -1;
-    for (int k = 0; k <= Dmax; ++k) prow[k] = 0, orow[k] = -1;
-    return;
-  }
-  const int A = best >> 20, astar = 0xFFFFF - (best & 0xFFFFF);
-  accept_len[b] = A;
-  int s = astar + 1;
-  for (int k = A; k >= 0; --k) {
-    prow[k] = s;
-    s = ps[s];
-  }
-  for (int k = A + 1; k <= Dmax; ++k) prow[k] = 0, orow[k] = -1;
-  for (int k = 0; k < A; ++k) orow[k] = tok[prow[k + 1] - 1];
-  orow[A] = s_tstar[astar];
+  __shared__ int32_t s_path[256];
+  acc::tree_accept_block(part, chunks, tokens, parent_s, num_nodes, root_key, Nmax, Dmax, status, accept_len, path,
+                         out_tokens, s_tstar, s_path, staged ? s_tstar + Nmax : nullptr,
+                         staged ? reinterpret_cast<float2*>(s_tstar + 3 * Nmax + 2) : nullptr);
 }
 
 // Greedy chain (T == 0): accept while the draft equals the target argmax.
@@ -185,14 +122,14 @@ __global__ void chain_greedy_decide(const float2* __restrict__ part, int chunks,
   if (b >= B) return;
   int j = K;
   for (int k = 0; k < K; ++k)
-    if (x[(size_t)b * K + k] != merge_argmax(part + ((size_t)b * (K + 1) + k) * chunks, chunks)) {
+    if (x[(size_t)b * K + k] != acc::merge_argmax(part + ((size_t)b * (K + 1) + k) * chunks, chunks)) {
       j = k;
       break;
     }
   accept_len[b] = j;
   int32_t* orow = out_tokens + (size_t)b * (K + 1);
   for (int k = 0; k < j; ++k) orow[k] = x[(size_t)b * K + k];
-  orow[j] = merge_argmax(part + ((size_t)b * (K + 1) + j) * chunks, chunks);
+  orow[j] = acc::merge_argmax(part + ((size_t)b * (K + 1) + j) * chunks, chunks);
   for (int k = j + 1; k <= K; ++k) orow[k] = -1;
 }
 
@@ -202,28 +139,39 @@ size_t accept_greedy_ws(int B, int Nmax, int V) {
   return (size_t)B * Nmax * num_chunks(V) * sizeof(float2);
 }
 
+tsd_status launch_row_argmax(const void* logits, tsd_dtype dtype, int V, int rows_per_seq, const int32_t* num_rows,
+                             int B, void* ws, cudaStream_t stream) {
+  if (B == 0 || rows_per_seq == 0) return TSD_OK;
+  const int chunks = num_chunks(V);
+  float2* part = reinterpret_cast<float2*>(ws);
+  dim3 grid(chunks, rows_per_seq, B);
+  if (dtype == TSD_BF16)
+    launch_pdl(row_argmax_chunks<__nv_bfloat16>, grid, dim3(kThreads), 0, stream,
+               reinterpret_cast<const __nv_bfloat16*>(logits), V, rows_per_seq, num_rows, chunks, part);
+  else
+    launch_pdl(row_argmax_chunks<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(logits), V,
+               rows_per_seq, num_rows, chunks, part);
+  return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+}
+
+int argmax_chunks(int V) { return num_chunks(V); }
+
 tsd_status launch_accept_greedy(const void* logits, tsd_dtype dtype, int V, const int32_t* tokens,
                                 const int32_t* parent_s, const int32_t* num_nodes, const int32_t* root_key, int B,
                                 int Nmax, int Dmax, int32_t* accept_len, int32_t* path, int32_t* out_tokens,
                                 void* ws, int32_t* status, cudaStream_t stream) {
   if (B == 0) return TSD_OK;
   const int chunks = num_chunks(V);
-  float2* part = reinterpret_cast<float2*>(ws);
-  if (Nmax > 0) {
-    dim3 grid(chunks, Nmax, B);
-    if (dtype == TSD_BF16)
-      launch_pdl(row_argmax_chunks<__nv_bfloat16>, grid, dim3(kThreads), 0, stream,
-                 reinterpret_cast<const __nv_bfloat16*>(logits), V, Nmax, num_nodes, chunks, part);
-    else
-      launch_pdl(row_argmax_chunks<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(logits), V,
-                 Nmax, num_nodes, chunks, part);
-    if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
-  }
-  const size_t smem = (size_t)(Nmax > 0 ? Nmax : 1) * sizeof(int32_t);
+  if (launch_row_argmax(logits, dtype, V, Nmax, num_nodes, B, ws, stream) != TSD_OK) return TSD_ERR_CUDA;
+  size_t smem = (size_t)(Nmax > 0 ? Nmax : 1) * sizeof(int32_t);
+  // parent slots and tokens (2 Nmax + 1 ints, padded to 8 bytes) and the argmax partials copied on chip
+  const size_t stage = (size_t)(2 * Nmax + 2) * sizeof(int32_t) + (size_t)Nmax * chunks * sizeof(float2);
+  const int staged = (Nmax & 1) == 0 && smem + stage <= 96 * 1024 ? 1 : 0;
+  if (staged) smem += stage;
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(tree_accept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  launch_pdl(tree_accept_kernel, dim3(B), dim3(kThreads), smem, stream, (const float2*)part, chunks, tokens, parent_s,
-             num_nodes, root_key, Nmax, Dmax, accept_len, path, out_tokens, (const int32_t*)status);
+  launch_pdl(tree_accept_kernel, dim3(B), dim3(kThreads), smem, stream, (const float2*)ws, chunks, tokens, parent_s,
+             num_nodes, root_key, Nmax, Dmax, accept_len, path, out_tokens, (const int32_t*)status, staged);
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }
 

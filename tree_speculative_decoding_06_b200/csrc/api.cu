@@ -235,4 +235,44 @@ tsd_status tsd_kv_commit_paged(void* k_pages, void* v_pages, int num_blocks, int
   return launch_kv_commit(a, S(stream));
 }
 
+tsd_status tsd_tree_accept_commit(const void* logits, tsd_dtype logits_dtype, int V, const int32_t* tokens,
+                                  const int32_t* parent_s, const int32_t* num_nodes, const int32_t* root_key, int B,
+                                  int Nmax, int Dmax, const tsd_kv_cache* cache, const void* k_tree,
+                                  const void* v_tree, int Hkv, int d, tsd_dtype kv_dtype, tsd_commit_mode mode,
+                                  int32_t* history, int history_cap, int32_t* history_len, int32_t* accept_len,
+                                  int32_t* path, int32_t* out_tokens, void* workspace, size_t ws_bytes,
+                                  int32_t* status, void* stream) {
+  // acceptance checks, as tsd_tree_accept_greedy
+  if (!dtype_ok(logits_dtype)) return TSD_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || B > 65535 || Nmax < 0 || Nmax > 65535 || V <= 0 || Dmax < 0 || Dmax > 255) return TSD_ERR_INVALID_ARG;
+  if ((long long)Nmax * 4 > 160 * 1024) return TSD_ERR_INVALID_ARG;
+  if (!cache) return TSD_ERR_INVALID_ARG;
+  // commit checks, as tsd_kv_commit[_paged]
+  CommitArgs a{};
+  a.k_cache = cache->k, a.v_cache = cache->v, a.prefix_len = cache->prefix_len, a.block_table = cache->block_table;
+  if (cache->block_table) {
+    if (!pow2(cache->block_size) || cache->block_size < 8 || cache->block_size > 256 || cache->max_blocks < 0 ||
+        cache->num_blocks < 0)
+      return TSD_ERR_INVALID_ARG;
+    if ((long long)cache->max_blocks * cache->block_size > 0x7fffffffLL) return TSD_ERR_INVALID_ARG;
+    a.max_blocks = cache->max_blocks, a.block_shift = log2i(cache->block_size), a.num_blocks = cache->num_blocks;
+    a.Lcap = cache->max_blocks * cache->block_size;
+  } else {
+    if (cache->Lmax < 0) return TSD_ERR_INVALID_ARG;
+    a.Lcap = cache->Lmax;
+  }
+  a.num_nodes = num_nodes, a.B = B, a.Nmax = Nmax, a.Hkv = Hkv, a.d = d, a.Dmax = Dmax, a.status = status;
+  // the path is produced in the kernel; commit_common only checks it is given in PATH / INPLACE
+  tsd_status e = commit_common(a, k_tree, v_tree, path, accept_len, kv_dtype, mode);
+  if (e != TSD_OK || B == 0) return e;
+  if (!accept_len || !path || !out_tokens || !status || !parent_s || (Nmax > 0 && (!logits || !tokens)))
+    return TSD_ERR_INVALID_ARG;
+  if (history && (history_cap < 0 || !history_len)) return TSD_ERR_INVALID_ARG;
+  const size_t need = tsd_tree_accept_greedy_workspace_size(B, Nmax, V);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return TSD_ERR_WORKSPACE;
+  SpliceArgs sp{history, history_cap, history_len};
+  return launch_accept_commit(logits, logits_dtype, V, tokens, parent_s, root_key, accept_len, path, out_tokens, a, sp,
+                              workspace, S(stream));
+}
+
 }  // extern "C"

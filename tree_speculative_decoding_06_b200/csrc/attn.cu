@@ -431,6 +431,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a, int BM,
 // ------------------------------------------------------------------------------------------
 // Split merge: o = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), one warp per query row.
 // ------------------------------------------------------------------------------------------
+constexpr int kFastSplits = 16;   // merges of up to this many splits load everything at once
+
 template <int D, typename OutT>
 __global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int splits, int Rmax) {
   pdl_trigger();
@@ -454,6 +456,37 @@ __global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int split
   const float* wo = reinterpret_cast<const float*>(a.workspace);
   const float* wml = wo + (size_t)a.B * a.Hkv * splits * Rmax * D;
   const size_t base = ((size_t)b * a.Hkv + g) * splits * Rmax + r;
+  if (v.nsplit <= kFastSplits) {
+    // every load is issued up front (lane s holds split s's (max, sum); each lane holds its four
+    // columns of every split's partial row), so the merge waits for one round trip to memory
+    float2 ml = make_float2(-INFINITY, 0.f);
+    if (lane < v.nsplit) ml = *reinterpret_cast<const float2*>(wml + (base + (size_t)lane * Rmax) * 2);
+    float ov[kFastSplits][D / 32];
+#pragma unroll
+    for (int s = 0; s < kFastSplits; ++s) {
+      const float* src = wo + (base + (size_t)s * Rmax) * D + lane;
+#pragma unroll
+      for (int e = 0; e < D / 32; ++e) ov[s][e] = s < v.nsplit ? src[32 * e] : 0.f;
+    }
+    const float M = warp_max(ml.x);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    const float w = lane < v.nsplit ? exp2f(ml.x - Mu) : 0.f;
+    const float lsum = warp_sum(ml.y * w);
+    float acc[D / 32];
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int s = 0; s < kFastSplits; ++s) {
+      const float ws = __shfl_sync(0xffffffffu, w, s);
+#pragma unroll
+      for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(ov[s][e], ws, acc[e]);
+    }
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) store_out(orow + lane + 32 * e, acc[e] * inv);
+    if (lrow && lane == 0) *lrow = (M + __log2f(lsum)) * kLn2;
+    return;
+  }
   // lane s holds split s's (max, sum): all of them are fetched at once, not one after another
   float M = -INFINITY;
   for (int s0 = 0; s0 < v.nsplit; s0 += 32) {

@@ -10,11 +10,15 @@
 //     box by block, the tree's K/V by node for one KV head) into separate rings: a K slot is
 //     released as soon as S = Q K^T has read it, a V slot after P V, so loads run several tiles
 //     ahead of the math;
-//   * one thread (warp 3) issues tcgen05.mma: S into one of two TMEM tiles (128 lanes x 64 fp32
-//     columns) and O += P V into one of two 128 x 128 fp32 TMEM accumulators, with descriptors
-//     built once and advanced by constants;
-//   * two softmax warpgroups take alternate tiles (even / odd), each with its own S tile, P
-//     buffer, O accumulator and running (max, sum) -- a split of the key range inside the CTA,
+//   * one thread (warp 3) issues tcgen05.mma: S into one of four TMEM tiles (128 lanes x 64 fp32
+//     columns; two per softmax warpgroup, so the tensor cores compute a warpgroup's next S while
+//     it is still exponentiating the current one) and O += P V into one of two 128 x 128 fp32
+//     TMEM accumulators, with descriptors built once and advanced by constants;
+//   * P never touches shared memory: the softmax writes it as bf16 over the first half of its S
+//     tile in TMEM and the P V product reads its A operand from there, so shared-memory
+//     bandwidth is left to the TMA writes and the K and V operand reads;
+//   * two softmax warpgroups take alternate tiles (even / odd), each with its own two S tiles,
+//     O accumulator and running (max, sum) -- a split of the key range inside the CTA,
 //     merged by log-sum-exp in the epilogue.  In a warpgroup each warp owns one TMEM lane
 //     quarter, one query row per thread: a row's 64 scores come out of TMEM with one tcgen05.ld,
 //     so its max and sum need no shuffles.  The ancestor mask is applied only on tree tiles (bits
@@ -43,11 +47,11 @@ using namespace umma;
 constexpr int kBM = 128, kBN = 64, kD = 128;
 constexpr int kThreadsU = 384;                    // 12 warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 256;         // O_w at 128*w, S_w at 256 + 64*w
+constexpr uint32_t kColO = 0, kColS = 256;         // O_w at 128*w; S of tile i at 256 + 64*(i%4)
+constexpr int kSBufs = 4;                          // S tiles in TMEM: two per softmax warpgroup
 constexpr uint32_t kHalf = kBN * 128;              // one 64-column half of a K or V tile: 8 KB
 constexpr uint32_t kSlot = 2 * kHalf;              // one K or V tile: 16 KB
 constexpr uint32_t kQBytes = kBM * 256;            // 32 KB
-constexpr uint32_t kPBytes = kBM * 128;            // 16 KB per softmax warpgroup
 constexpr int kMaxRing = 6;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -58,14 +62,14 @@ struct UParams {
   int ks, vs;          // K and V ring depths
   int box_rows;        // rows per TMA box of the cache (64 contiguous, min(block, 64) paged)
   int W;               // ancestor-bit words per node
-  uint32_t k_off, v_off, p_off, mask_off;   // shared-memory offsets
+  uint32_t k_off, v_off, mask_off;   // shared-memory offsets
 };
 
 struct __align__(8) Bars {
   uint64_t q_full;
   uint64_t k_full[kMaxRing], k_empty[kMaxRing];
   uint64_t v_full[kMaxRing], v_empty[kMaxRing];
-  uint64_t s_full[2];    // warpgroup w: its S tile is in TMEM
+  uint64_t s_full[kSBufs];  // S tile of key tile i (buffer i % 4) is in TMEM
   uint64_t p_full[2];    // warpgroup w: its P tile is in shared memory (and its S tile was read)
   uint64_t pv_done[2];   // warpgroup w: its last P V product finished (P buffer free, O current)
   uint64_t fin;
@@ -77,6 +81,27 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
+
+// 2^x on the FMA pipe, for the lean full-tile path (finite x <= 8): x = j + f with j = round(x),
+// found by adding 1.5 * 2^23 (j then sits in the low mantissa bits), and f in [-0.5, 0.5].  2^f
+// is a cubic whose coefficients were fitted here for least maximum relative error on that
+// interval (7.5e-5, well below the bf16 rounding that P gets before P V), and j is added to the
+// exponent field.  x below -125 is clamped there (2^-125 instead of a smaller number: no effect
+// on a row whose largest term is 2^0 or more).  The multi-function unit has 1/8 of the FMA
+// pipe's lanes, so taking some exponentials off it shortens the softmax (the split of work
+// between the two units follows "FlashAttention-4", which emulates part of exp2 in software on
+// Blackwell for the same reason).
+__device__ __forceinline__ float poly_exp2(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+// Of each group of four exponentials in a full tile, this many are computed by poly_exp2.  Measured
+// on B200: 1 of 4 made the MUFU-heavy forest case 18% slower and 2 of 4 40% slower -- the softmax
+// warps are bound by instruction issue, not by the multi-function unit -- so it is 0 for now.
+constexpr int kPolyPerQuad = 0;
 
 __device__ __forceinline__ void abort_cta(const AttnArgs& a, int b, volatile int* s_abort) {
   if (*s_abort == 0) {
@@ -176,7 +201,6 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   uint8_t* sQ = smem;
   uint8_t* sK = smem + u.k_off;
   uint8_t* sV = smem + u.v_off;
-  uint8_t* sP = smem + u.p_off;
   uint32_t* sMask = reinterpret_cast<uint32_t*>(smem + u.mask_off);
 
   // ---------------------------------------------------------------- set-up
@@ -184,8 +208,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < u.ks; ++s) mbar_init(&bars.k_full[s], 1), mbar_init(&bars.k_empty[s], 1);
     for (int s = 0; s < u.vs; ++s) mbar_init(&bars.v_full[s], 1), mbar_init(&bars.v_empty[s], 1);
+    for (int sb = 0; sb < kSBufs; ++sb) mbar_init(&bars.s_full[sb], 1);
     for (int w = 0; w < 2; ++w) {
-      mbar_init(&bars.s_full[w], 1);
       mbar_init(&bars.p_full[w], 4);
       mbar_init(&bars.pv_done[w], 1);
     }
@@ -262,40 +286,40 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     const uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dk = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t dv = sdesc_sw128(smem_u32(sV), kHalf, 1024);
-    const uint64_t dp = sdesc_sw128(smem_u32(sP), 16, 1024);
-    bool ok = mbar_wait(&bars.q_full, 0);
+    // every lane waits and the verdict is made warp-uniform: the MMA issue below is
+    // warp-collective (elect.sync) and needs the whole warp converged
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
+    };
+    bool ok = wait_all(&bars.q_full, 0);
     int k_consumed = 0, v_consumed = 0;
-    // S(j) = Q K(j)^T into warpgroup (j & 1)'s S tile; frees the K slot when done
+    // S(j) = Q K(j)^T into S buffer j % 4 (warpgroup j & 1); frees the K slot when done
     auto issue_s = [&](int j) -> bool {
       const int st = j % u.ks;
-      if (!mbar_wait(&bars.k_full[st], (j / u.ks) & 1)) return false;
+      if (!wait_all(&bars.k_full[st], (j / u.ks) & 1)) return false;
       ++k_consumed;
-      if (lane == 0) {
-        tc_fence_after();
-        const uint64_t bk = dk + (uint64_t)((st * kSlot) >> 4);
-        const uint32_t d = tmem + kColS + (uint32_t)(j & 1) * kBN;
+      tc_fence_after();
+      const uint64_t bk = dk + (uint64_t)((st * kSlot) >> 4);
+      const uint32_t d = tmem + kColS + (uint32_t)(j % kSBufs) * kBN;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off_q = ((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4;
-          const uint32_t off_k = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(d, dq + off_q, bk + off_k, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bars.k_empty[st]);
-        tc_commit(&bars.s_full[j & 1]);
+      for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint32_t off_q = ((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4;
+        const uint32_t off_k = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+        mma_bf16_ss_warp(d, dq + off_q, bk + off_k, idesc_s, kk > 0 ? 1u : 0u);
       }
-      __syncwarp();
+      tc_commit_warp(&bars.k_empty[st]);
+      tc_commit_warp(&bars.s_full[j % kSBufs]);
       return true;
     };
-    if (ok && nt > 0) ok = issue_s(0);
-    if (ok && nt > 1) ok = issue_s(1);
+    for (int j = 0; ok && j < kSBufs && j < nt; ++j) ok = issue_s(j);
     for (int i = 0; ok && i < nt; ++i) {
       const int w = i & 1;
-      if (!mbar_wait(&bars.p_full[w], (i >> 1) & 1)) {
+      if (!wait_all(&bars.p_full[w], (i >> 1) & 1)) {
         ok = false;
         break;
       }
       const int st = i % u.vs;
-      if (!mbar_wait(&bars.v_full[st], (i / u.vs) & 1)) {
+      if (!wait_all(&bars.v_full[st], (i / u.vs) & 1)) {
         ok = false;
         break;
       }
@@ -313,19 +337,16 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         fence_proxy_async();
       }
       __syncwarp();
-      if (lane == 0) {
-        tc_fence_after();
-        const uint64_t bv = dv + (uint64_t)((st * kSlot) >> 4);
-        const uint64_t ap = dp + (uint64_t)((w * kPBytes) >> 4);
-        const uint32_t d = tmem + kColO + (uint32_t)w * kD;
+      tc_fence_after();
+      const uint64_t bv = dv + (uint64_t)((st * kSlot) >> 4);
+      const uint32_t ap = tmem + kColS + (uint32_t)(i % kSBufs) * kBN;   // P(i) over S(i)
+      const uint32_t d = tmem + kColO + (uint32_t)w * kD;
 #pragma unroll
-        for (int kb = 0; kb < kBN / 16; ++kb)
-          mma_bf16_ss(d, ap + (uint32_t)(kb * 2), bv + (uint32_t)(kb * 128), idesc_o, (i >= 2 || kb > 0) ? 1u : 0u);
-        tc_commit(&bars.v_empty[st]);
-        tc_commit(&bars.pv_done[w]);
-      }
-      __syncwarp();
-      if (i + 2 < nt) ok = issue_s(i + 2);   // warpgroup w has read its S tile: it can be reused
+      for (int kb = 0; kb < kBN / 16; ++kb)
+        mma_bf16_ts_warp(d, ap + (uint32_t)(kb * 8), bv + (uint32_t)(kb * 128), idesc_o, (i >= 2 || kb > 0) ? 1u : 0u);
+      tc_commit_warp(&bars.v_empty[st]);
+      tc_commit_warp(&bars.pv_done[w]);
+      if (i + kSBufs < nt) ok = issue_s(i + kSBufs);   // warpgroup w has read S(i): its buffer is free
     }
     if (!ok) abort_cta(a, b, &s_abort);
     if (lane == 0) s_k_consumed = k_consumed, s_v_consumed = v_consumed;
@@ -341,14 +362,14 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     const bool warp_live = r0 + q4 * 32 < r_hi;
     const int nl = row / G;
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-    const uint32_t s_col = kColS + (uint32_t)wg * kBN, o_col = kColO + (uint32_t)wg * kD;
+    const uint32_t o_col = kColO + (uint32_t)wg * kD;
     const float sl2 = a.scale * kLog2e;
-    uint8_t* sPw = sP + (size_t)wg * kPBytes;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = wg; i < nt; i += 2) {
       const int k = i >> 1;
-      if (!mbar_wait(&bars.s_full[wg], k & 1)) {
+      const uint32_t s_col = kColS + (uint32_t)(i % kSBufs) * kBN;
+      if (!mbar_wait(&bars.s_full[i % kSBufs], (i / kSBufs) & 1)) {
         ok = false;
         break;
       }
@@ -365,7 +386,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         tmem_ld32(lane_addr + s_col + 32, s1);
         tmem_wait_ld();
         float mx;
-        if (!tree && kbase + kBN <= v.L) {
+        const bool full = !tree && kbase + kBN <= v.L;
+        if (full) {
           // a full prefix tile: every key is visible to every row, no mask work
           float ma[8];
 #pragma unroll
@@ -411,6 +433,22 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         }
         const float nmu = m_used == -INFINITY ? 0.f : -m_used;
         float suma[4] = {0.f, 0.f, 0.f, 0.f};
+        if (full) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float x0 = fmaf(__uint_as_float(s0[c]), sl2, nmu);
+            const float x1 = fmaf(__uint_as_float(s0[c + 1]), sl2, nmu);
+            const float x2 = fmaf(__uint_as_float(s1[c]), sl2, nmu);
+            const float x3 = fmaf(__uint_as_float(s1[c + 1]), sl2, nmu);
+            const float p0 = kPolyPerQuad >= 4 ? poly_exp2(x0) : fast_exp2(x0);
+            const float p1 = kPolyPerQuad >= 3 ? poly_exp2(x1) : fast_exp2(x1);
+            const float p2 = kPolyPerQuad >= 2 ? poly_exp2(x2) : fast_exp2(x2);
+            const float p3 = kPolyPerQuad >= 1 ? poly_exp2(x3) : fast_exp2(x3);
+            suma[(c >> 1) & 3] += (p0 + p1) + (p2 + p3);
+            pk[c / 2] = pack_bf16x2(p0, p1);
+            pk[16 + c / 2] = pack_bf16x2(p2, p3);
+          }
+        } else {
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           // p = 2^(s * scale * log2(e) - m): one FFMA feeds the exponential (masked s = -inf gives 0)
@@ -422,9 +460,10 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           pk[c / 2] = pack_bf16x2(p0, p1);
           pk[16 + c / 2] = pack_bf16x2(p2, p3);
         }
+        }
         l = l * alpha + ((suma[0] + suma[1]) + (suma[2] + suma[3]));
       }
-      // this warpgroup's previous P V (tile i - 2) must be done: P buffer free, O up to date
+      // this warpgroup's previous P V (tile i - 2) must be done before O is rescaled
       if (k >= 1 && !mbar_wait(&bars.pv_done[wg], (k - 1) & 1)) {
         ok = false;
         break;
@@ -442,14 +481,10 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         }
         tmem_wait_st();
       }
-      if (warp_live) {   // P row -> swizzled shared tile (row = TMEM lane)
-        uint8_t* prow = sPw + (size_t)row * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      if (warp_live) {   // P row (bf16 pairs) over the first 32 columns of its S tile
+        tmem_st32(lane_addr + s_col, pk);
+        tmem_wait_st();
       }
-      fence_proxy_async();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full[wg]);
@@ -600,9 +635,9 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   u.W = (a.Nmax + 31) / 32;
   const uint32_t mask_bytes = (uint32_t)(kBM / G) * u.W * 4;
   auto total = [&](int ks, int vs) {
-    return 1024 + kQBytes + (uint32_t)(ks + vs) * kSlot + 2 * kPBytes + mask_bytes;
+    return 1024 + kQBytes + (uint32_t)(ks + vs) * kSlot + mask_bytes;
   };
-  u.ks = 5, u.vs = 4;   // K is consumed first (by S = Q K^T), so its ring runs further ahead
+  u.ks = 6, u.vs = 5;   // K is consumed first (by S = Q K^T), so its ring runs further ahead
   const uint32_t limit = 227 * 1024 - 2048;   // leave room for the static shared variables
   while (total(u.ks, u.vs) > limit && u.vs > 2) {
     if (u.ks > u.vs) --u.ks; else --u.vs;
@@ -610,8 +645,7 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   if (total(u.ks, u.vs) > limit) return TSD_ERR_INVALID_ARG;
   u.k_off = kQBytes;
   u.v_off = u.k_off + (uint32_t)u.ks * kSlot;
-  u.p_off = u.v_off + (uint32_t)u.vs * kSlot;
-  u.mask_off = u.p_off + 2 * kPBytes;
+  u.mask_off = u.v_off + (uint32_t)u.vs * kSlot;
   const size_t smem = total(u.ks, u.vs);
 
   CUtensorMap mq, mk, mv, mkt, mvt;

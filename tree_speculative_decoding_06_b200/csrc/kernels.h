@@ -108,6 +108,22 @@ struct CommitArgs {
 };
 tsd_status launch_kv_commit(const CommitArgs& a, cudaStream_t stream);
 
+// Vocabulary argmax scan of rows_per_seq rows per sequence into ws (float2 per (row, chunk)).
+tsd_status launch_row_argmax(const void* logits, tsd_dtype dtype, int V, int rows_per_seq, const int32_t* num_rows,
+                             int B, void* ws, cudaStream_t stream);
+int argmax_chunks(int V);
+// Greedy tree acceptance fused with the commit of the accepted path (and an optional splice of
+// the emitted tokens into a device token history).  a.accept_len / a.path are unused.
+struct SpliceArgs {
+  int32_t* history;      // [B, cap] or null
+  int cap;
+  int32_t* history_len;  // [B]
+};
+tsd_status launch_accept_commit(const void* logits, tsd_dtype dtype, int V, const int32_t* tokens,
+                                const int32_t* parent_s, const int32_t* root_key, int32_t* accept_len,
+                                int32_t* path, int32_t* out_tokens, const CommitArgs& a, const SpliceArgs& sp,
+                                void* ws, cudaStream_t stream);
+
 int device_sm_count();
 
 }  // namespace tsd

@@ -7,7 +7,9 @@
 //
 // One CTA per sequence; one thread per node.  Each node's check depends only on its own parent
 // and its ancestors, so the first offending node (smallest index) is found with an atomicMin on
-// (node << 4 | code): if every node below it is valid, its own verdict is exact.
+// (node << 4 | code): if every node below it is valid, its own verdict is exact.  The parent
+// array is first copied into shared memory with one coalesced read (when it fits), so the
+// ancestor walks are chains of shared-memory loads rather than of dependent global loads.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -16,12 +18,18 @@ namespace tsd {
 __global__ void tree_prepare_kernel(const int32_t* __restrict__ parent, const int32_t* __restrict__ num_nodes,
                                     int Nmax, int Dmax, int forest, int32_t* __restrict__ parent_s,
                                     int32_t* __restrict__ depth_s, int32_t* __restrict__ anc,
-                                    uint32_t* __restrict__ anc_bits, int32_t* __restrict__ status) {
+                                    uint32_t* __restrict__ anc_bits, int32_t* __restrict__ status, int staged) {
   pdl_trigger();
   pdl_wait();
+  extern __shared__ int32_t s_par[];
   const int b = blockIdx.x;
   const int N = num_nodes ? num_nodes[b] : Nmax;
   const int32_t* par = parent + (size_t)b * Nmax;
+  if (staged) {
+    const int n = (N >= 0 && N <= Nmax) ? N : 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s_par[i] = par[i];
+    par = s_par;   // made visible by the __syncthreads below
+  }
   const int S = Nmax + 1;                  // slots per sequence
   const int AW = Dmax + 1;                 // ancestor-table width
   const int W = (S + 31) >> 5;             // ancestor-bit words per slot
@@ -100,8 +108,10 @@ tsd_status launch_tree_prepare(const int32_t* parent, const int32_t* num_nodes, 
                                int32_t* status, cudaStream_t stream) {
   if (B == 0) return TSD_OK;
   const int threads = Nmax + 1 >= 256 ? 256 : ((Nmax + 1 + 31) / 32) * 32;
-  if (launch_pdl(tree_prepare_kernel, dim3(B), dim3(threads), 0, stream, parent, num_nodes, Nmax, Dmax, forest, parent_s,
-                 depth, anc, anc_bits, status) != cudaSuccess)
+  const size_t smem = (size_t)Nmax * sizeof(int32_t);
+  const int staged = smem <= 48 * 1024 ? 1 : 0;
+  if (launch_pdl(tree_prepare_kernel, dim3(B), dim3(threads), staged ? smem : 0, stream, parent, num_nodes, Nmax, Dmax,
+                 forest, parent_s, depth, anc, anc_bits, status, staged) != cudaSuccess)
     return TSD_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }

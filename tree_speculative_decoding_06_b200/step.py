@@ -3,11 +3,14 @@
 ``VerifyStep(...)`` sizes every output and workspace for one batch shape; ``run(inputs)``
 enqueues, on the current stream and without any host synchronisation,
 
-    tsd_tree_prepare -> tsd_tree_verify_attn[_paged] -> tsd_tree_accept_greedy
-    (or tsd_chain_accept_sample for a linear draft) -> tsd_kv_commit[_paged]
+    tsd_tree_prepare -> tsd_tree_verify_attn[_paged] -> tsd_tree_accept_commit
+    (greedy acceptance and the commit of its path in one call; with fused=False the two
+    separate calls tsd_tree_accept_greedy -> tsd_kv_commit[_paged])
+    or, for a linear draft, tsd_chain_accept_sample -> tsd_kv_commit[_paged] (length mode)
 
 and returns the device tensors it wrote.  The cache and prefix_len in `inputs` are updated in
-place by the commit, exactly as a decoding loop would carry them into the next step.
+place by the commit, exactly as a decoding loop would carry them into the next step; with
+history_cap > 0 the emitted tokens are also appended to a device token history.
 """
 from __future__ import annotations
 
@@ -16,7 +19,7 @@ from typing import Optional
 import torch
 
 from . import (tree_prepare, tree_verify_attn, tree_verify_attn_paged, tree_accept_greedy, chain_accept_sample,
-               kv_commit, kv_commit_paged, tree_verify_attn_workspace_size, tree_verify_attn_paged_workspace_size,
+               kv_commit, kv_commit_paged, tree_accept_commit, tree_verify_attn_workspace_size, tree_verify_attn_paged_workspace_size,
                tree_accept_greedy_workspace_size, chain_accept_sample_workspace_size, TSD_BF16, TSD_F32)
 
 
@@ -24,9 +27,11 @@ class VerifyStep:
     def __init__(self, *, B: int, Nmax: int, Hq: int, Hkv: int, d: int, Dmax: int, V: int, dtype: torch.dtype,
                  Lmax: Optional[int] = None, paged: bool = False, block_size: int = 16,
                  max_blocks: Optional[int] = None, forest: bool = False, accept: str = "greedy", K: int = 0,
-                 device="cuda"):
+                 fused: bool = True, history_cap: int = 0, T: float = 0.0, device="cuda"):
         self.B, self.Nmax, self.Hq, self.Hkv, self.d, self.Dmax, self.V = B, Nmax, Hq, Hkv, d, Dmax, V
         self.dtype, self.paged, self.forest, self.accept, self.K = dtype, paged, forest, accept, K
+        self.fused = fused and accept == "greedy"
+        self.T = T
         dt = TSD_BF16 if dtype == torch.bfloat16 else TSD_F32
         dev = torch.device(device)
         i32 = dict(dtype=torch.int32, device=dev)
@@ -52,6 +57,17 @@ class VerifyStep:
             self.accept_len = torch.zeros(B, **i32)
             self.path = None
             self.out_tokens = torch.zeros(B, K + 1, **i32)
+        self.history = torch.zeros(B, history_cap, **i32) if history_cap > 0 and self.fused else None
+        self.history_len = torch.zeros(B, **i32) if self.history is not None else None
+        self.splits_merge = ws > 0
+
+    def launches_per_step(self) -> int:
+        """Kernels one run() launches: prepare, attention (+ split merge), acceptance (scan +
+        decide, or the chain sampler's three), commit (inside the fused acceptance)."""
+        n = 2 + int(self.splits_merge)
+        if self.accept == "greedy":
+            return n + (2 if self.fused else 3)
+        return n + (3 if self.T > 0 else 2) + 1
 
     def run(self, x: dict) -> dict:
         tree_prepare(x["parent"], x.get("num_nodes"), self.Dmax, self.forest, parent_s=self.parent_s,
@@ -64,6 +80,18 @@ class VerifyStep:
             tree_verify_attn(x["q"], x["k_cache"], x["v_cache"], x["prefix_len"], x.get("k_tree"), x.get("v_tree"),
                              self.parent_s, x.get("num_nodes"), self.Dmax, out=self.out, workspace=self.attn_ws,
                              status=self.status)
+        if self.fused:
+            if self.paged:
+                kc, vc, bt = x["k_pages"], x["v_pages"], x["block_table"]
+            else:
+                kc, vc, bt = x["k_cache"], x["v_cache"], None
+            tree_accept_commit(x["logits"], x["tokens"], self.parent_s, kc, vc, x["prefix_len"], x["k_tree"],
+                               x["v_tree"], x.get("num_nodes"), x.get("root_key"), self.Dmax, "path",
+                               block_table=bt, history=self.history, history_len=self.history_len,
+                               accept_len=self.accept_len, path=self.path, out_tokens=self.out_tokens,
+                               workspace=self.acc_ws, status=self.status)
+            return {"out": self.out, "accept_len": self.accept_len, "path": self.path,
+                    "out_tokens": self.out_tokens, "status": self.status, "parent_s": self.parent_s}
         if self.accept == "greedy":
             tree_accept_greedy(x["logits"], x["tokens"], self.parent_s, x.get("num_nodes"), x.get("root_key"),
                                self.Dmax, accept_len=self.accept_len, path=self.path, out_tokens=self.out_tokens,
@@ -83,7 +111,7 @@ class VerifyStep:
                 "status": self.status, "parent_s": self.parent_s}
 
     @staticmethod
-    def for_inputs(x: dict, device="cuda") -> "VerifyStep":
+    def for_inputs(x: dict, device="cuda", **kw) -> "VerifyStep":
         """Size a step for a device input dict as produced by ``to_device``."""
         B, Nmax, Hq, d = x["q"].shape
         Hkv = x["k_tree"].shape[2]
@@ -94,7 +122,8 @@ class VerifyStep:
                           Lmax=None if paged else x["k_cache"].shape[2], paged=paged,
                           block_size=x["k_pages"].shape[2] if paged else 16,
                           max_blocks=x["block_table"].shape[1] if paged else None, forest=bool(x.get("forest")),
-                          accept=accept, K=(x["z_p"].shape[1] - 1) if accept == "sample" else 0, device=device)
+                          accept=accept, K=(x["z_p"].shape[1] - 1) if accept == "sample" else 0, device=device,
+                          T=float(x.get("T", 0.0)) if accept == "sample" else 0.0, **kw)
 
 
 def to_device(inp: dict, device="cuda") -> dict:
