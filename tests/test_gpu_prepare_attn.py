@@ -144,9 +144,10 @@ def test_attention_capacity_flag():
     assert (out[1] == 0).all()
 
 
-def test_no_cross_branch_leakage_gpu():
+@pytest.mark.parametrize("Hq", [8, 16])   # 104 query rows per KV head (one tile), 208 (two tiles)
+def test_no_cross_branch_leakage_gpu(Hq):
     parent = W.tree_static_scored((4, 3, 2, 1, 1, 1), 26)
-    inp = W.make_custom_inputs([parent], [150], Hq=8, Hkv=2, d=128, dtype="bf16", seed=11)
+    inp = W.make_custom_inputs([parent], [150], Hq=Hq, Hkv=2, d=128, dtype="bf16", seed=11)
     out0, _, _ = gpu_attention(inp)
     M = oracle.tree_structure(parent, 6)["M"]
     rng = np.random.default_rng(1)

@@ -555,7 +555,12 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
   if (p.BM <= 0) p.BM = 16;
   p.mtiles = (p.Rmax + p.BM - 1) / p.BM;
   p.max_tiles = (Lcap + p.BN - 1) / p.BN + (Nmax + p.BN - 1) / p.BN;
-  const long long base = (long long)B * Hkv * p.mtiles;
+  // the tcgen05 kernel (bf16, d = 128, power-of-two groups) takes two 128-row query tiles per CTA
+  // when a KV head has more than 128 query rows, streaming each K/V tile once for both
+  const bool umma_shape = dtype == TSD_BF16 && d == 128 && p.G <= 128 && (p.G & (p.G - 1)) == 0;
+  p.dual = umma_shape && p.Rmax > 128;
+  p.umtiles = p.dual ? (p.Rmax + 255) / 256 : p.mtiles;
+  const long long base = (long long)B * Hkv * (umma_shape ? p.umtiles : p.mtiles);
   const int sms = device_sm_count();
   // Split count: the CTAs of one launch run in waves of one CTA per SM, a CTA costs its tiles plus a
   // fixed overhead (set-up, pipeline fill, epilogue) of about two tiles, and every split adds

@@ -49,6 +49,9 @@ constexpr int kThreadsU = 384;                    // 12 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256;         // O_w at 128*w; S of tile i at 256 + 64*(i%4)
 constexpr int kSBufs = 4;                          // S tiles in TMEM: two per softmax warpgroup
+// Two-query-tile CTAs: S_w at 256 + 64*w (one per warpgroup) and the query tile Q_w itself at
+// 384 + 64*w (bf16 pairs), the A operand of S = Q K^T read from TMEM instead of shared memory.
+constexpr uint32_t kColQ = 384;
 constexpr uint32_t kHalf = kBN * 128;              // one 64-column half of a K or V tile: 8 KB
 constexpr uint32_t kSlot = 2 * kHalf;              // one K or V tile: 16 KB
 constexpr uint32_t kQBytes = kBM * 256;            // 32 KB
@@ -163,6 +166,10 @@ __device__ __forceinline__ void load_tile(const AttnArgs& a, const SeqView& v, c
   }
 }
 
+// kDual: the CTA owns two 128-row query tiles of the same KV head and streams every K/V tile once
+// for both (warpgroup w owns query tile w over all key tiles); otherwise one query tile whose key
+// tiles alternate between the two warpgroups.
+template <bool kDual>
 __global__ void __launch_bounds__(kThreadsU, 1)
     attn_umma_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
@@ -183,9 +190,10 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   const int g = blockIdx.y, b = blockIdx.z;
   const int G = a.Hq / a.Hkv;
   const SeqView v = seq_view(a, b, G, kBN, u.tps);
-  const int r0 = mt * kBM;
+  constexpr int kRows = kDual ? 2 * kBM : kBM;   // query rows of this CTA
+  const int r0 = mt * kRows;
   if (v.skip || r0 >= v.R) return;
-  const int r_hi = min(r0 + kBM, v.R);
+  const int r_hi = min(r0 + kRows, v.R);
   if (v.zero) {
     if (split == 0) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
     if (split == 0 && mt == 0 && g == 0 && tid == 0 && a.status[b] == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
@@ -195,7 +203,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   const bool direct = (v.nsplit == 1);
   const int t_begin = split * u.tps;
   const int nt = min(v.T, t_begin + u.tps) - t_begin;
-  const int nodes_per_tile = kBM / G;
+  const int nodes_per_tile = kRows / G;
   const int node0 = mt * nodes_per_tile;
 
   uint8_t* sQ = smem;
@@ -205,7 +213,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
-    mbar_init(&bars.q_full, 1);
+    mbar_init(&bars.q_full, kDual ? 8 : 1);   // two query tiles: each softmax warp stores its rows
     for (int s = 0; s < u.ks; ++s) mbar_init(&bars.k_full[s], 1), mbar_init(&bars.k_empty[s], 1);
     for (int s = 0; s < u.vs; ++s) mbar_init(&bars.v_full[s], 1), mbar_init(&bars.v_empty[s], 1);
     for (int sb = 0; sb < kSBufs; ++sb) mbar_init(&bars.s_full[sb], 1);
@@ -236,10 +244,12 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ K producer (one thread), Q first
     if (lane == 0) {
-      mbar_expect_tx(&bars.q_full, kQBytes);
-      const int zq = b * a.Nmax + node0;
-      tma_load_3d(sQ, &tmQ, 0, g * G, zq, &bars.q_full);
-      tma_load_3d(sQ + kQBytes / 2, &tmQ, 64, g * G, zq, &bars.q_full);
+      if (!kDual) {
+        mbar_expect_tx(&bars.q_full, kQBytes);
+        const int zq = b * a.Nmax + node0;
+        tma_load_3d(sQ, &tmQ, 0, g * G, zq, &bars.q_full);
+        tma_load_3d(sQ + kQBytes / 2, &tmQ, 64, g * G, zq, &bars.q_full);
+      }
       int issued = 0;
       TileBlocks nxt;
       fetch_blocks(a, v, u, b, t_begin, nxt);
@@ -311,6 +321,75 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       tc_commit_warp(&bars.s_full[j % kSBufs]);
       return true;
     };
+    // zero V rows past the valid keys of a partial tile (its TMA box may hold stale rows)
+    auto zero_v_tail = [&](int i, int st) {
+      const int t = t_begin + i;
+      const int nv = t < v.nPT ? min(kBN, v.L - t * kBN) : min(kBN, v.N - (t - v.nPT) * kBN);
+      if (nv < kBN) {
+        uint8_t* dV = sV + (size_t)st * kSlot;
+        const int nchunks = (kBN - nv) * 8;   // 16-byte chunks per half
+        for (int c = lane; c < 2 * nchunks; c += 32) {
+          const int half = c / nchunks, cc = c % nchunks;
+          *reinterpret_cast<uint4*>(dV + half * kHalf + (size_t)nv * 128 + (size_t)cc * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();
+      }
+      __syncwarp();
+    };
+    if constexpr (kDual) {
+      // S_w(j) = Q_w K(j)^T into warpgroup w's S tile, A = Q_w from TMEM (8 columns per k-step);
+      // the K slot is freed after both
+      auto issue_s_w = [&](int j, int w) -> bool {
+        const int st = j % u.ks;
+        if (w == 0) {
+          if (!wait_all(&bars.k_full[st], (j / u.ks) & 1)) return false;
+          ++k_consumed;
+        }
+        tc_fence_after();
+        const uint64_t bk = dk + (uint64_t)((st * kSlot) >> 4);
+        const uint32_t aq = tmem + kColQ + (uint32_t)w * 64;
+        const uint32_t d = tmem + kColS + (uint32_t)w * kBN;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off_k = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          mma_bf16_ts_warp(d, aq + (uint32_t)(kk * 8), bk + off_k, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        if (w == 1) tc_commit_warp(&bars.k_empty[st]);
+        tc_commit_warp(&bars.s_full[w]);
+        return true;
+      };
+      if (ok && nt > 0) {
+        ok = issue_s_w(0, 0);
+        if (ok) ok = issue_s_w(0, 1);
+      }
+      for (int i = 0; ok && i < nt; ++i) {
+        const int st = i % u.vs;
+        if (!wait_all(&bars.v_full[st], (i / u.vs) & 1)) {
+          ok = false;
+          break;
+        }
+        ++v_consumed;
+        zero_v_tail(i, st);
+        const uint64_t bv = dv + (uint64_t)((st * kSlot) >> 4);
+        for (int w = 0; ok && w < 2; ++w) {
+          if (!wait_all(&bars.p_full[w], i & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ap = tmem + kColS + (uint32_t)w * kBN;   // P_w(i) over S_w(i)
+          const uint32_t d = tmem + kColO + (uint32_t)w * kD;
+#pragma unroll
+          for (int kb = 0; kb < kBN / 16; ++kb)
+            mma_bf16_ts_warp(d, ap + (uint32_t)(kb * 8), bv + (uint32_t)(kb * 128), idesc_o, (i > 0 || kb > 0) ? 1u : 0u);
+          if (w == 1) tc_commit_warp(&bars.v_empty[st]);
+          tc_commit_warp(&bars.pv_done[w]);
+          // S_w(i+1) overwrites P_w(i): tcgen05.mma of one thread execute in issue order, so the
+          // P V product just issued has read its A operand first
+          if (i + 1 < nt) ok = issue_s_w(i + 1, w);
+        }
+      }
+    } else {
     for (int j = 0; ok && j < kSBufs && j < nt; ++j) ok = issue_s(j);
     for (int i = 0; ok && i < nt; ++i) {
       const int w = i & 1;
@@ -324,19 +403,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         break;
       }
       ++v_consumed;
-      // zero V rows past the valid keys of a partial tile (its TMA box may hold stale rows)
-      const int t = t_begin + i;
-      const int nv = t < v.nPT ? min(kBN, v.L - t * kBN) : min(kBN, v.N - (t - v.nPT) * kBN);
-      if (nv < kBN) {
-        uint8_t* dV = sV + (size_t)st * kSlot;
-        const int nchunks = (kBN - nv) * 8;   // 16-byte chunks per half
-        for (int c = lane; c < 2 * nchunks; c += 32) {
-          const int half = c / nchunks, cc = c % nchunks;
-          *reinterpret_cast<uint4*>(dV + half * kHalf + (size_t)nv * 128 + (size_t)cc * 16) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async();
-      }
-      __syncwarp();
+      zero_v_tail(i, st);
       tc_fence_after();
       const uint64_t bv = dv + (uint64_t)((st * kSlot) >> 4);
       const uint32_t ap = tmem + kColS + (uint32_t)(i % kSBufs) * kBN;   // P(i) over S(i)
@@ -348,28 +415,53 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       tc_commit_warp(&bars.pv_done[w]);
       if (i + kSBufs < nt) ok = issue_s(i + kSBufs);   // warpgroup w has read S(i): its buffer is free
     }
+    }
     if (!ok) abort_cta(a, b, &s_abort);
     if (lane == 0) s_k_consumed = k_consumed, s_v_consumed = v_consumed;
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax warpgroups
     const int wg = (warp - 4) >> 2;
     const int q4 = warp & 3;                       // TMEM lane quarter of this warp
-    const int row = q4 * 32 + lane;
-    const int r = r0 + row;
+    const int row = q4 * 32 + lane;                // TMEM lane = row of the query tile
+    const int qrow = (kDual ? wg * kBM : 0) + row;  // row within the CTA's query rows
+    const int r = r0 + qrow;
     const bool row_ok = r < r_hi;
     // a warp whose 32 rows are all padding skips the softmax; its P rows are never read into an
     // output row (each output row depends on its own P row only)
-    const bool warp_live = r0 + q4 * 32 < r_hi;
-    const int nl = row / G;
+    const bool warp_live = r0 + qrow - lane < r_hi;
+    const int nl = qrow / G;
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
     const uint32_t o_col = kColO + (uint32_t)wg * kD;
     const float sl2 = a.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int i = wg; i < nt; i += 2) {
-      const int k = i >> 1;
-      const uint32_t s_col = kColS + (uint32_t)(i % kSBufs) * kBN;
-      if (!mbar_wait(&bars.s_full[i % kSBufs], (i / kSBufs) & 1)) {
+    if constexpr (kDual) {
+      // this thread's query row into TMEM as bf16 pairs (64 columns of Q_w): the A operand of
+      // S = Q K^T; rows past the sequence's rows are zero
+      const int i_node = r / G, hh = r % G;
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                                                        (((size_t)b * a.Nmax + (row_ok ? i_node : 0)) * a.Hq +
+                                                         g * G + hh) * kD);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t qv[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 x = row_ok ? src[half * 8 + c] : make_uint4(0, 0, 0, 0);
+          qv[4 * c] = x.x, qv[4 * c + 1] = x.y, qv[4 * c + 2] = x.z, qv[4 * c + 3] = x.w;
+        }
+        tmem_st32(lane_addr + kColQ + (uint32_t)wg * 64 + (uint32_t)half * 32, qv);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.q_full);
+    }
+    for (int i = kDual ? 0 : wg; i < nt; i += kDual ? 1 : 2) {
+      const int k = kDual ? i : i >> 1;            // this warpgroup's k-th tile
+      const int buf = kDual ? wg : wg + 2 * (k & 1);
+      const uint32_t s_col = kColS + (uint32_t)buf * kBN;
+      if (!mbar_wait(&bars.s_full[buf], kDual ? (k & 1) : ((k >> 1) & 1))) {
         ok = false;
         break;
       }
@@ -490,11 +582,12 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       if (lane == 0) mbar_arrive(&bars.p_full[wg]);
     }
     // the warpgroup's last P V product
-    if (ok && nt > wg && !mbar_wait(&bars.pv_done[wg], ((nt - 1 - wg) >> 1) & 1)) ok = false;
+    const int kn = kDual ? nt : (nt - wg + 1) >> 1;   // tiles this warpgroup processed
+    if (ok && kn > 0 && !mbar_wait(&bars.pv_done[wg], (kn - 1) & 1)) ok = false;
     if (!ok) abort_cta(a, b, &s_abort);
     row_m = m_used;
     row_l = l;
-    if (wg == 1) s_ml1[row] = make_float2(m_used, l);
+    if (!kDual && wg == 1) s_ml1[row] = make_float2(m_used, l);
   }
 
   // ---------------------------------------------------------------- epilogue / teardown
@@ -502,18 +595,22 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   __syncthreads();
   tc_fence_after();
   if (!s_abort) {
-    if (warp >= 4 && warp < 8) {
-      // merge the two warpgroups' partial results of this row (log-sum-exp), then write it
+    if (kDual ? warp >= 4 : (warp >= 4 && warp < 8)) {
+      // one query tile: merge the two warpgroups' partial results of this row (log-sum-exp);
+      // two query tiles: each warpgroup holds its rows' complete result.  Then write the row.
+      const int wg = (warp - 4) >> 2;
       const int q4 = warp & 3;
       const int row = q4 * 32 + lane;
-      const int r = r0 + row;
+      const int r = r0 + (kDual ? wg * kBM : 0) + row;
       const bool row_ok = r < r_hi;
       const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-      const float2 ml1 = nt > 1 ? s_ml1[row] : make_float2(-INFINITY, 0.f);
+      const uint32_t o_first = kColO + (kDual ? (uint32_t)wg * kD : 0u);
+      const bool two = !kDual && nt > 1;   // a second accumulator (warpgroup 1's) to merge
+      const float2 ml1 = two ? s_ml1[row] : make_float2(-INFINITY, 0.f);
       const float M = fmaxf(row_m, ml1.x);
       const float Mu = M == -INFINITY ? 0.f : M;
       const float a0 = exp2f(row_m - Mu);
-      const float a1 = nt > 1 ? exp2f(ml1.x - Mu) : 0.f;
+      const float a1 = two ? exp2f(ml1.x - Mu) : 0.f;
       const float l = row_l * a0 + ml1.y * a1;
       const bool err = s_err != 0;
       const int i_node = r / G, hh = r % G;
@@ -525,13 +622,13 @@ __global__ void __launch_bounds__(kThreadsU, 1)
 #pragma unroll
         for (int ch = 0; ch < kD / 32; ++ch) {
           uint32_t o0[32], o1[32];
-          tmem_ld32(lane_addr + kColO + ch * 32, o0);
-          if (nt > 1) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
+          tmem_ld32(lane_addr + o_first + ch * 32, o0);
+          if (two) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
           tmem_wait_ld();
           float f[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            f[e] = __uint_as_float(o0[e]) * c0 + (nt > 1 ? __uint_as_float(o1[e]) * c1 : 0.f);
+            f[e] = __uint_as_float(o0[e]) * c0 + (two ? __uint_as_float(o1[e]) * c1 : 0.f);
           if (row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
@@ -550,8 +647,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
 #pragma unroll
         for (int ch = 0; ch < kD / 32; ++ch) {
           uint32_t o0[32], o1[32];
-          tmem_ld32(lane_addr + kColO + ch * 32, o0);
-          if (nt > 1) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
+          tmem_ld32(lane_addr + o_first + ch * 32, o0);
+          if (two) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
           tmem_wait_ld();
           if (row_ok) {
             float4* dst = reinterpret_cast<float4*>(wo + (base + r) * kD + ch * 32);
@@ -560,7 +657,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
               float f[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                f[e] = __uint_as_float(o0[4 * q + e]) * a0 + (nt > 1 ? __uint_as_float(o1[4 * q + e]) * a1 : 0.f);
+                f[e] = __uint_as_float(o0[4 * q + e]) * a0 + (two ? __uint_as_float(o1[4 * q + e]) * a1 : 0.f);
               dst[q] = make_float4(f[0], f[1], f[2], f[3]);
             }
           }
@@ -631,11 +728,13 @@ bool umma_eligible(const AttnArgs& a, tsd_dtype dtype) {
 tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   UParams u{};
-  u.tps = p.tps, u.splits = p.splits, u.Rmax = p.Rmax, u.mtiles = p.mtiles;
+  u.tps = p.tps, u.splits = p.splits, u.Rmax = p.Rmax, u.mtiles = p.umtiles;
+  const int rows = p.dual ? 2 * kBM : kBM;   // query rows per CTA
+  const uint32_t q_bytes = p.dual ? 0u : kQBytes;   // two query tiles live in TMEM, not shared memory
   u.W = (a.Nmax + 31) / 32;
-  const uint32_t mask_bytes = (uint32_t)(kBM / G) * u.W * 4;
+  const uint32_t mask_bytes = (uint32_t)(rows / G) * u.W * 4;
   auto total = [&](int ks, int vs) {
-    return 1024 + kQBytes + (uint32_t)(ks + vs) * kSlot + mask_bytes;
+    return 1024 + q_bytes + (uint32_t)(ks + vs) * kSlot + mask_bytes;
   };
   u.ks = 6, u.vs = 5;   // K is consumed first (by S = Q K^T), so its ring runs further ahead
   const uint32_t limit = 227 * 1024 - 2048;   // leave room for the static shared variables
@@ -643,7 +742,7 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
     if (u.ks > u.vs) --u.ks; else --u.vs;
   }
   if (total(u.ks, u.vs) > limit) return TSD_ERR_INVALID_ARG;
-  u.k_off = kQBytes;
+  u.k_off = q_bytes;
   u.v_off = u.k_off + (uint32_t)u.ks * kSlot;
   u.mask_off = u.v_off + (uint32_t)u.vs * kSlot;
   const size_t smem = total(u.ks, u.vs);
@@ -678,9 +777,10 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
     if (!make_map(&mkt, a.k_tree, 3, dims, str, box) || !make_map(&mvt, a.v_tree, 3, dims, str, box))
       return TSD_ERR_CUDA;
   }
-  cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  dim3 grid(p.mtiles * p.splits, a.Hkv, a.B);
-  if (launch_pdl(attn_umma_kernel, grid, dim3(kThreadsU), smem, stream, mq, mk, mv, mkt, mvt, a, u) != cudaSuccess)
+  auto kernel = p.dual ? attn_umma_kernel<true> : attn_umma_kernel<false>;
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid(u.mtiles * p.splits, a.Hkv, a.B);
+  if (launch_pdl(kernel, grid, dim3(kThreadsU), smem, stream, mq, mk, mv, mkt, mvt, a, u) != cudaSuccess)
     return TSD_ERR_CUDA;
   return TSD_OK;
 }

@@ -39,6 +39,8 @@ struct AttnPlan {
   int BN = 64;              // keys per tile
   int max_tiles = 0;        // prefix tiles at capacity + tree tiles
   int tps = 1, splits = 1;  // tiles per split, splits per (sequence, KV head, row tile)
+  bool dual = false;        // tcgen05 kernel: two 128-row query tiles per CTA
+  int umtiles = 0;          // tcgen05 kernel: CTAs per (sequence, KV head, split)
   int threads = 128;
   size_t smem = 0;
   size_t ws_bytes = 0;
