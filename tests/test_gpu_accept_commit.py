@@ -288,14 +288,15 @@ def test_commit_errors_leave_cache_untouched():
 
 
 # ----------------------------------------------------------------------------- whole step
-@pytest.mark.parametrize("name", ["tiny", "tree26", "eagle60", "chain5", "forest"])
-def test_verify_step_matches_oracle(name):
+@pytest.mark.parametrize("name,schedule", [(n, s) for n in ("tiny", "tree26", "eagle60", "forest")
+                                            for s in ("overlap", "fused", "serial")] + [("chain5", None)])
+def test_verify_step_matches_oracle(name, schedule):
     w = W.WORKLOADS[name]
     if name in ("chain5", "forest", "eagle60"):
         w = w.scaled(B=min(w.B, 4), L=min(w.L, 3000), L_lo=None if w.L_lo is None else 500)
     inp = W.make_inputs(w, nan_guard=False)
     x = to_device(inp)
-    step = VerifyStep.for_inputs(x)
+    step = VerifyStep.for_inputs(x, schedule=schedule)
     res = step.run(x)
     torch.cuda.synchronize()
     assert (res["status"].cpu().numpy() == 0).all()

@@ -132,21 +132,37 @@ def test_fused_flagged_sequence_is_skipped():
     assert np.array_equal(pl, rpl) and np.array_equal(kc, rk)
 
 
-@pytest.mark.parametrize("paged", [False, True])
-def test_device_resident_loop(paged):
+@pytest.mark.parametrize("paged,schedule,graph", [(False, "fused", False), (True, "fused", False),
+                                                  (False, "overlap", False), (True, "overlap", True),
+                                                  (False, "fused", True)])
+def test_device_resident_loop(paged, schedule, graph):
     """Three verify steps back to back with nothing read back in between: each step's commit
     advances prefix_len on the device and the next step's attention reads the grown cache.
-    Every step is checked against the oracle applied to the cache the previous step left."""
+    Every step is checked against the oracle applied to the cache the previous step left.  With
+    graph=True the three steps are captured into one CUDA graph and replayed once."""
     parents = [W.tree_static_scored((4, 3, 2, 1, 1, 1), 26), W.tree_chain(4)]
     inp = W.make_custom_inputs(parents, [40, 75], Hq=8, Hkv=2, d=128, dtype="bf16", seed=5, paged=paged,
                                nan_guard=False, plant_p=0.9)
     x = to_device(inp)
-    step = VerifyStep.for_inputs(x, history_cap=64)
-    outs = []
-    for _ in range(3):
-        res = step.run(x)
-        outs.append({"out": res["out"].clone(), "accept_len": res["accept_len"].clone(),
-                     "out_tokens": res["out_tokens"].clone()})
+    fused = schedule == "fused"
+    step = VerifyStep.for_inputs(x, schedule=schedule, history_cap=64 if fused else 0)
+    outs = [{"out": torch.empty_like(step.out), "accept_len": torch.empty_like(step.accept_len),
+             "out_tokens": torch.empty_like(step.out_tokens)} for _ in range(3)]
+
+    def three_steps():
+        for o in outs:
+            res = step.run(x)
+            for k in o:
+                o[k].copy_(res[k])
+
+    if graph:
+        s = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            three_steps()
+        g.replay()
+    else:
+        three_steps()
     torch.cuda.synchronize()
     assert (step.status.cpu().numpy() == 0).all()
     cur = dict(inp)
@@ -168,7 +184,8 @@ def test_device_resident_loop(paged):
         cur[key], cur[vkey], cur["prefix_len"] = rk, rv, rpl
     assert np.array_equal(x["prefix_len"].cpu().numpy(), cur["prefix_len"])
     assert np.array_equal(_cache_np(x[key]), cur[key]) and np.array_equal(_cache_np(x[vkey]), cur[vkey])
-    hl = step.history_len.cpu().numpy()
-    h = step.history.cpu().numpy()
-    for b in range(2):
-        assert hl[b] == len(hist[b]) and h[b, :hl[b]].tolist() == hist[b]
+    if fused:
+        hl = step.history_len.cpu().numpy()
+        h = step.history.cpu().numpy()
+        for b in range(2):
+            assert hl[b] == len(hist[b]) and h[b, :hl[b]].tolist() == hist[b]

@@ -26,6 +26,28 @@ __device__ __forceinline__ int merge_argmax(const float2* p, int chunks) {
   return bi == INT_MAX ? 0 : bi;
 }
 
+// Warp-parallel merge of the chunk partials of rows [0, n) held in shared memory (chunks <= 32):
+// one row per warp at a time, lane c holds chunk c, a shuffle tree keeps the best (ties -> lower
+// index).  Writes s_tstar[row].
+__device__ __forceinline__ void merge_rows_warp(const float2* s_part, int chunks, int n, int32_t* s_tstar) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int r = warp; r < n; r += nw) {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    if (lane < chunks) {
+      const float2 p = s_part[(size_t)r * chunks + lane];
+      bv = p.x, bi = __float_as_int(p.y);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (better(ov, oi, bv, bi)) bv = ov, bi = oi;
+    }
+    if (lane == 0) s_tstar[r] = bi == INT_MAX ? 0 : bi;
+  }
+}
+
 // Acceptance of sequence b by the whole CTA.  s_tstar holds >= Nmax ints of shared memory;
 // s_stage, if not null, >= 2 * Nmax + 1 more, into which the tree's parent slots and tokens are
 // copied first (one coalesced read each) so that the ancestor walks run on shared memory;
@@ -65,7 +87,12 @@ __device__ __forceinline__ int tree_accept_block(const float2* __restrict__ part
     const float2* src = part + (size_t)b * Nmax * chunks;
     for (int k = threadIdx.x; k < Nmax * chunks; k += blockDim.x) s_part[k] = src[k];
     __syncthreads();
-    for (int i = threadIdx.x; live && i < N; i += blockDim.x) s_tstar[i] = merge_argmax(s_part + (size_t)i * chunks, chunks);
+    if (chunks <= 32) {
+      if (live) merge_rows_warp(s_part, chunks, N, s_tstar);
+    } else {
+      for (int i = threadIdx.x; live && i < N; i += blockDim.x)
+        s_tstar[i] = merge_argmax(s_part + (size_t)i * chunks, chunks);
+    }
   } else {
     for (int i = threadIdx.x; live && i < N; i += blockDim.x)
       s_tstar[i] = merge_argmax(part + ((size_t)b * Nmax + i) * chunks, chunks);
@@ -99,29 +126,34 @@ __device__ __forceinline__ int tree_accept_block(const float2* __restrict__ part
     if (ok) atomicMax(&s_best, (d << 20) | (0xFFFFF - i));
   }
   __syncthreads();
+  // thread 0 walks the path into shared memory; then every thread writes its entries
   if (threadIdx.x == 0) {
     const int best = live ? s_best : -1;
     if (best < 0) {
-      accept_len[b] = -1;
-      for (int k = 0; k <= Dmax; ++k) prow[k] = 0, orow[k] = -1;
       s_A = -1;
     } else {
       const int A = best >> 20, astar = 0xFFFFF - (best & 0xFFFFF);
-      accept_len[b] = A;
       int s = astar + 1;
       for (int k = A; k >= 0; --k) {
-        prow[k] = s;
         s_path[k] = s;
         s = ps[s];
       }
-      for (int k = A + 1; k <= Dmax; ++k) prow[k] = 0, orow[k] = -1;
-      for (int k = 0; k < A; ++k) orow[k] = tok[s_path[k + 1] - 1];
-      orow[A] = s_tstar[astar];
       s_A = A;
     }
   }
   __syncthreads();
-  return s_A;
+  const int A = s_A;
+  if (threadIdx.x == 0) accept_len[b] = A;
+  for (int k = threadIdx.x; k <= Dmax; k += blockDim.x) {
+    if (k <= A) {
+      prow[k] = s_path[k];
+      orow[k] = k < A ? tok[s_path[k + 1] - 1] : s_tstar[s_path[A] - 1];
+    } else {
+      prow[k] = 0;
+      orow[k] = -1;
+    }
+  }
+  return A;
 }
 
 }  // namespace acc

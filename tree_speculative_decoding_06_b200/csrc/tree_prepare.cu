@@ -25,9 +25,8 @@ __global__ void tree_prepare_kernel(const int32_t* __restrict__ parent, const in
   const int b = blockIdx.x;
   const int N = num_nodes ? num_nodes[b] : Nmax;
   const int32_t* par = parent + (size_t)b * Nmax;
-  if (staged) {
-    const int n = (N >= 0 && N <= Nmax) ? N : 0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) s_par[i] = par[i];
+  if (staged) {   // all Nmax entries (in bounds whatever N is): the copy need not wait for N
+    for (int i = threadIdx.x; i < Nmax; i += blockDim.x) s_par[i] = par[i];
     par = s_par;   // made visible by the __syncthreads below
   }
   const int S = Nmax + 1;                  // slots per sequence

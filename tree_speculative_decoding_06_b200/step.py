@@ -3,10 +3,15 @@
 ``VerifyStep(...)`` sizes every output and workspace for one batch shape; ``run(inputs)``
 enqueues, on the current stream and without any host synchronisation,
 
-    tsd_tree_prepare -> tsd_tree_verify_attn[_paged] -> tsd_tree_accept_commit
-    (greedy acceptance and the commit of its path in one call; with fused=False the two
-    separate calls tsd_tree_accept_greedy -> tsd_kv_commit[_paged])
-    or, for a linear draft, tsd_chain_accept_sample -> tsd_kv_commit[_paged] (length mode)
+    tsd_tree_prepare -> tsd_tree_verify_attn[_paged] -> acceptance -> tsd_kv_commit[_paged]
+
+The greedy acceptance depends on the tree and the target logits only, not on the attention, so by
+default (schedule "overlap") it runs on a second stream forked after prepare -- the vocabulary scan
+and the acceptance then use the SMs the attention leaves idle -- and the commit (which must follow
+the attention: it advances prefix_len, which the attention reads) joins both.  Schedule "fused"
+runs tsd_tree_accept_commit after the attention on one stream (and can splice the emitted tokens
+into a device token history); "serial" runs tsd_tree_accept_greedy then tsd_kv_commit on one
+stream.  A linear draft takes tsd_chain_accept_sample -> tsd_kv_commit[_paged] (length mode).
 
 and returns the device tensors it wrote.  The cache and prefix_len in `inputs` are updated in
 place by the commit, exactly as a decoding loop would carry them into the next step; with
@@ -27,10 +32,19 @@ class VerifyStep:
     def __init__(self, *, B: int, Nmax: int, Hq: int, Hkv: int, d: int, Dmax: int, V: int, dtype: torch.dtype,
                  Lmax: Optional[int] = None, paged: bool = False, block_size: int = 16,
                  max_blocks: Optional[int] = None, forest: bool = False, accept: str = "greedy", K: int = 0,
-                 fused: bool = True, history_cap: int = 0, T: float = 0.0, device="cuda"):
+                 schedule: Optional[str] = None, history_cap: int = 0, T: float = 0.0, device="cuda"):
         self.B, self.Nmax, self.Hq, self.Hkv, self.d, self.Dmax, self.V = B, Nmax, Hq, Hkv, d, Dmax, V
         self.dtype, self.paged, self.forest, self.accept, self.K = dtype, paged, forest, accept, K
-        self.fused = fused and accept == "greedy"
+        if accept != "greedy":
+            schedule = "serial"
+        elif schedule is None:
+            schedule = "fused" if history_cap > 0 else "overlap"
+        if schedule not in ("overlap", "fused", "serial"):
+            raise ValueError(f"unknown schedule {schedule!r}")
+        if history_cap > 0 and schedule != "fused":
+            raise ValueError("a token history needs the fused schedule")
+        self.schedule = schedule
+        self.fused = schedule == "fused"
         self.T = T
         dt = TSD_BF16 if dtype == torch.bfloat16 else TSD_F32
         dev = torch.device(device)
@@ -60,6 +74,9 @@ class VerifyStep:
         self.history = torch.zeros(B, history_cap, **i32) if history_cap > 0 and self.fused else None
         self.history_len = torch.zeros(B, **i32) if self.history is not None else None
         self.splits_merge = ws > 0
+        if schedule == "overlap":
+            self.side = torch.cuda.Stream(device=dev)
+            self.ev_fork, self.ev_join = torch.cuda.Event(), torch.cuda.Event()
 
     def launches_per_step(self) -> int:
         """Kernels one run() launches: prepare, attention (+ split merge), acceptance (scan +
@@ -69,9 +86,21 @@ class VerifyStep:
             return n + (2 if self.fused else 3)
         return n + (3 if self.T > 0 else 2) + 1
 
+    def _accept(self, x: dict):
+        tree_accept_greedy(x["logits"], x["tokens"], self.parent_s, x.get("num_nodes"), x.get("root_key"),
+                           self.Dmax, accept_len=self.accept_len, path=self.path, out_tokens=self.out_tokens,
+                           workspace=self.acc_ws, status=self.status)
+
     def run(self, x: dict) -> dict:
         tree_prepare(x["parent"], x.get("num_nodes"), self.Dmax, self.forest, parent_s=self.parent_s,
                      depth=self.depth, anc=self.anc, status=self.status)
+        if self.schedule == "overlap":   # acceptance on the side stream, concurrently with the attention
+            main = torch.cuda.current_stream(self.parent_s.device)
+            self.ev_fork.record(main)
+            self.side.wait_event(self.ev_fork)
+            with torch.cuda.stream(self.side):
+                self._accept(x)
+                self.ev_join.record(self.side)
         if self.paged:
             tree_verify_attn_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["prefix_len"],
                                    x.get("k_tree"), x.get("v_tree"), self.parent_s, x.get("num_nodes"), self.Dmax,
@@ -93,9 +122,10 @@ class VerifyStep:
             return {"out": self.out, "accept_len": self.accept_len, "path": self.path,
                     "out_tokens": self.out_tokens, "status": self.status, "parent_s": self.parent_s}
         if self.accept == "greedy":
-            tree_accept_greedy(x["logits"], x["tokens"], self.parent_s, x.get("num_nodes"), x.get("root_key"),
-                               self.Dmax, accept_len=self.accept_len, path=self.path, out_tokens=self.out_tokens,
-                               workspace=self.acc_ws, status=self.status)
+            if self.schedule == "overlap":
+                main.wait_event(self.ev_join)
+            else:
+                self._accept(x)
             mode = "path"
         else:
             chain_accept_sample(x["z_p"], x["z_q"], x["x"], x["u"], x["T"], accept_len=self.accept_len,
