@@ -83,6 +83,28 @@ __device__ __forceinline__ void build_mask(const AttnArgs& a, int b, int i_lo, i
   }
 }
 
+// build_mask by one warp from a shared-memory copy of the sequence's parent slots (s_ps holds
+// N + 1 ints): one coalesced read, then the ancestor walks are chains of shared-memory loads.
+__device__ __forceinline__ void build_mask_staged(const AttnArgs& a, int b, int i_lo, int cnt, int W, uint32_t* smask,
+                                                  int N, int32_t* s_ps, int lane) {
+  const int32_t* ps = a.parent_s + (size_t)b * (a.Nmax + 1);
+  for (int s = lane; s <= N; s += 32) s_ps[s] = ps[s];
+  __syncwarp();
+  for (int n = lane; n < cnt; n += 32) {
+    uint32_t* row = smask + (size_t)n * W;
+    for (int w = 0; w < W; ++w) row[w] = 0u;
+    if (i_lo + n >= N) continue;
+    int s = i_lo + n + 1;
+    for (int step = 0; step <= a.Dmax && s != 0; ++step) {
+      const int j = s - 1;
+      row[j >> 5] |= 1u << (j & 31);
+      const int p = s_ps[s];
+      if (p >= s || p < 0) break;   // prepare rejects such trees; never walk upward-out-of-range
+      s = p;
+    }
+  }
+}
+
 template <typename OutT>
 __device__ __forceinline__ void store_out(OutT* o, float v);
 template <>

@@ -52,6 +52,10 @@ constexpr int kSBufs = 4;                          // S tiles in TMEM: two per s
 // Two-query-tile CTAs: S_w at 256 + 64*w (one per warpgroup) and the query tile Q_w itself at
 // 384 + 64*w (bf16 pairs), the A operand of S = Q K^T read from TMEM instead of shared memory.
 constexpr uint32_t kColQ = 384;
+// Epilogue staging rows in shared memory (the K/V rings are idle by then), padded by 16 bytes so
+// that the 32 rows a warp writes at once spread over all banks.
+constexpr uint32_t kStageF = kD * 4 + 16;   // fp32 split partial row
+constexpr uint32_t kStageH = kD * 2 + 16;   // bf16 output row
 constexpr uint32_t kHalf = kBN * 128;              // one 64-column half of a K or V tile: 8 KB
 constexpr uint32_t kSlot = 2 * kHalf;              // one K or V tile: 16 KB
 constexpr uint32_t kQBytes = kBM * 256;            // 32 KB
@@ -65,7 +69,8 @@ struct UParams {
   int ks, vs;          // K and V ring depths
   int box_rows;        // rows per TMA box of the cache (64 contiguous, min(block, 64) paged)
   int W;               // ancestor-bit words per node
-  uint32_t k_off, v_off, mask_off;   // shared-memory offsets
+  int stage;           // epilogue rows go through shared memory (the ring region is large enough)
+  uint32_t k_off, v_off, mask_off, ps_off;   // shared-memory offsets
 };
 
 struct __align__(8) Bars {
@@ -75,6 +80,7 @@ struct __align__(8) Bars {
   uint64_t s_full[kSBufs];  // S tile of key tile i (buffer i % 4) is in TMEM
   uint64_t p_full[2];    // warpgroup w: its P tile is in shared memory (and its S tile was read)
   uint64_t pv_done[2];   // warpgroup w: its last P V product finished (P buffer free, O current)
+  uint64_t mask_full;    // the ancestor bits of the tree tiles are in shared memory
   uint64_t fin;
 };
 
@@ -221,6 +227,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       mbar_init(&bars.p_full[w], 4);
       mbar_init(&bars.pv_done[w], 1);
     }
+    mbar_init(&bars.mask_full, 1);
     mbar_init(&bars.fin, 1);
     s_err = 0;
     s_abort = 0;
@@ -231,9 +238,6 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   if (warp == 3) {
     tmem_alloc(&s_tmem, kTmemCols);
     tmem_relinquish();
-  }
-  if (warp == 1) {
-    if (t_begin + nt > v.nPT) build_mask(a, b, node0, nodes_per_tile, u.W, sMask, v.N, lane, 32);
   }
   tc_fence_before();
   __syncthreads();
@@ -266,6 +270,15 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         ++issued;
       }
       s_k_issued = issued;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ ancestor bits of the tree tiles
+    // built while the first prefix tiles stream in; the softmax waits for them at its first tree tile
+    if (t_begin + nt > v.nPT) {
+      build_mask_staged(a, b, node0, nodes_per_tile, u.W, sMask, v.N, reinterpret_cast<int32_t*>(smem + u.ps_off),
+                        lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.mask_full);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ V producer (one thread)
@@ -435,6 +448,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     const float sl2 = a.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    bool mask_ready = false;
     if constexpr (kDual) {
       // this thread's query row into TMEM as bf16 pairs (64 columns of Q_w): the A operand of
       // S = Q K^T; rows past the sequence's rows are zero
@@ -492,6 +506,13 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         } else {
           const int lim = tree ? v.N : v.L;
           uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
+          if (tree && !mask_ready) {
+            if (!mbar_wait(&bars.mask_full, 0)) {
+              ok = false;
+              break;
+            }
+            mask_ready = true;
+          }
           if (tree) {
             const int wi = kbase >> 5;
             w0 = sMask[nl * u.W + wi];
@@ -594,6 +615,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  uint8_t* sStage = smem + u.k_off;   // the K/V rings, idle once every P V product is done
+  if (!s_abort && u.stage) fence_proxy_async();   // last read there by the tensor cores
   if (!s_abort) {
     if (kDual ? warp >= 4 : (warp >= 4 && warp < 8)) {
       // one query tile: merge the two warpgroups' partial results of this row (log-sum-exp);
@@ -601,7 +624,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       const int wg = (warp - 4) >> 2;
       const int q4 = warp & 3;
       const int row = q4 * 32 + lane;
-      const int r = r0 + (kDual ? wg * kBM : 0) + row;
+      const int crow = (kDual ? wg * kBM : 0) + row;   // row within this CTA's rows
+      const int r = r0 + crow;
       const bool row_ok = r < r_hi;
       const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
       const uint32_t o_first = kColO + (kDual ? (uint32_t)wg * kD : 0u);
@@ -630,7 +654,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           for (int e = 0; e < 32; ++e)
             f[e] = __uint_as_float(o0[e]) * c0 + (two ? __uint_as_float(o1[e]) * c1 : 0.f);
           if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+            uint4* dst = u.stage ? reinterpret_cast<uint4*>(sStage + (size_t)crow * kStageH + ch * 64)
+                                 : reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               dst[q] = make_uint4(pack_bf16x2(f[8 * q], f[8 * q + 1]), pack_bf16x2(f[8 * q + 2], f[8 * q + 3]),
@@ -651,7 +676,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           if (two) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
           tmem_wait_ld();
           if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(wo + (base + r) * kD + ch * 32);
+            float4* dst = u.stage ? reinterpret_cast<float4*>(sStage + (size_t)crow * kStageF + ch * 128)
+                                  : reinterpret_cast<float4*>(wo + (base + r) * kD + ch * 32);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               float f[4];
@@ -665,6 +691,28 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         if (row_ok) *reinterpret_cast<float2*>(wml + (base + r) * 2) = make_float2(M, l);
       }
       if (err && split == 0 && mt == 0 && g == 0 && tid == 128) flag_status(a.status, b, TSD_ERR_CAPACITY);
+    }
+    if (u.stage) {
+      // every thread copies staged rows out with coalesced 16-byte stores
+      __syncthreads();
+      const int nrows = r_hi - r0;
+      if (direct) {
+        for (int idx = tid; idx < nrows * (kD / 8); idx += kThreadsU) {
+          const int cr = idx / (kD / 8), c = idx % (kD / 8);
+          const int rr = r0 + cr, node = rr / G, hh = rr % G;
+          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                (((size_t)b * a.Nmax + node) * a.Hq + g * G + hh) * kD;
+          reinterpret_cast<uint4*>(orow)[c] = *reinterpret_cast<const uint4*>(sStage + (size_t)cr * kStageH + c * 16);
+        }
+      } else {
+        float* wo = reinterpret_cast<float*>(a.workspace);
+        const size_t base = (((size_t)b * a.Hkv + g) * u.splits + split) * u.Rmax + r0;
+        for (int idx = tid; idx < nrows * (kD / 4); idx += kThreadsU) {
+          const int cr = idx / (kD / 4), c = idx % (kD / 4);
+          reinterpret_cast<float4*>(wo + (base + cr) * kD)[c] =
+              *reinterpret_cast<const float4*>(sStage + (size_t)cr * kStageF + c * 16);
+        }
+      }
     }
   } else {
     // time-out: let this CTA's own TMA copies and MMAs land (bounded) before freeing TMEM
@@ -733,8 +781,9 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   const uint32_t q_bytes = p.dual ? 0u : kQBytes;   // two query tiles live in TMEM, not shared memory
   u.W = (a.Nmax + 31) / 32;
   const uint32_t mask_bytes = (uint32_t)(rows / G) * u.W * 4;
+  const uint32_t ps_bytes = (uint32_t)(a.Nmax + 1) * 4;   // the tree's parent slots, staged for the mask
   auto total = [&](int ks, int vs) {
-    return 1024 + q_bytes + (uint32_t)(ks + vs) * kSlot + mask_bytes;
+    return 1024 + q_bytes + (uint32_t)(ks + vs) * kSlot + ((mask_bytes + 15) & ~15u) + ps_bytes;
   };
   u.ks = 6, u.vs = 5;   // K is consumed first (by S = Q K^T), so its ring runs further ahead
   const uint32_t limit = 227 * 1024 - 2048;   // leave room for the static shared variables
@@ -745,6 +794,8 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   u.k_off = q_bytes;
   u.v_off = u.k_off + (uint32_t)u.ks * kSlot;
   u.mask_off = u.v_off + (uint32_t)u.vs * kSlot;
+  u.ps_off = u.mask_off + ((mask_bytes + 15) & ~15u);
+  u.stage = (uint32_t)(u.ks + u.vs) * kSlot >= (uint32_t)rows * kStageF ? 1 : 0;
   const size_t smem = total(u.ks, u.vs);
 
   CUtensorMap mq, mk, mv, mkt, mvt;
