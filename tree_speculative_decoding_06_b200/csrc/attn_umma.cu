@@ -107,6 +107,37 @@ __device__ __forceinline__ float poly_exp2(float x) {
   const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
+// Paired fp32 arithmetic of sm_100 (one instruction for two lanes of work) and the three-input
+// maximum: the lean full-tile softmax issues a third fewer instructions with them.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0, float c1) {
+  asm("{\n"
+      ".reg .b64 ra, rb, rc, rd;\n"
+      "mov.b64 ra, {%2, %3};\n"
+      "mov.b64 rb, {%4, %5};\n"
+      "mov.b64 rc, {%6, %7};\n"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n"
+      "mov.b64 {%0, %1}, rd;\n"
+      "}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n"
+      ".reg .b64 ra, rb, rd;\n"
+      "mov.b64 ra, {%2, %3};\n"
+      "mov.b64 rb, {%4, %5};\n"
+      "add.rn.f32x2 rd, ra, rb;\n"
+      "mov.b64 {%0, %1}, rd;\n"
+      "}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Of each group of four exponentials in a full tile, this many are computed by poly_exp2.  Measured
 // on B200: 1 of 4 made the MUFU-heavy forest case 18% slower and 2 of 4 40% slower -- the softmax
 // warps are bound by instruction issue, not by the multi-function unit -- so it is 0 for now.
@@ -499,9 +530,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
 #pragma unroll
           for (int q = 0; q < 8; ++q) ma[q] = fmaxf(__uint_as_float(s0[q]), __uint_as_float(s1[q]));
 #pragma unroll
-          for (int c = 8; c < 32; ++c)
-            ma[c & 7] = fmaxf(ma[c & 7], fmaxf(__uint_as_float(s0[c]), __uint_as_float(s1[c])));
-          mx = fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
+          for (int c = 8; c < 32; ++c) ma[c & 7] = max3f(ma[c & 7], __uint_as_float(s0[c]), __uint_as_float(s1[c]));
+          mx = max3f(max3f(ma[0], ma[1], ma[2]), max3f(ma[3], ma[4], ma[5]), fmaxf(ma[6], ma[7]));
           mx = row_ok ? mx * sl2 : -INFINITY;
         } else {
           const int lim = tree ? v.N : v.L;
@@ -548,16 +578,17 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         float suma[4] = {0.f, 0.f, 0.f, 0.f};
         if (full) {
 #pragma unroll
+          // pair sums: suma[0..1] gather the even/odd keys of s0, suma[2..3] those of s1
           for (int c = 0; c < 32; c += 2) {
-            const float x0 = fmaf(__uint_as_float(s0[c]), sl2, nmu);
-            const float x1 = fmaf(__uint_as_float(s0[c + 1]), sl2, nmu);
-            const float x2 = fmaf(__uint_as_float(s1[c]), sl2, nmu);
-            const float x3 = fmaf(__uint_as_float(s1[c + 1]), sl2, nmu);
+            float x0, x1, x2, x3;
+            fma2(x0, x1, __uint_as_float(s0[c]), __uint_as_float(s0[c + 1]), sl2, sl2, nmu, nmu);
+            fma2(x2, x3, __uint_as_float(s1[c]), __uint_as_float(s1[c + 1]), sl2, sl2, nmu, nmu);
             const float p0 = kPolyPerQuad >= 4 ? poly_exp2(x0) : fast_exp2(x0);
             const float p1 = kPolyPerQuad >= 3 ? poly_exp2(x1) : fast_exp2(x1);
             const float p2 = kPolyPerQuad >= 2 ? poly_exp2(x2) : fast_exp2(x2);
             const float p3 = kPolyPerQuad >= 1 ? poly_exp2(x3) : fast_exp2(x3);
-            suma[(c >> 1) & 3] += (p0 + p1) + (p2 + p3);
+            add2(suma[0], suma[1], suma[0], suma[1], p0, p1);
+            add2(suma[2], suma[3], suma[2], suma[3], p2, p3);
             pk[c / 2] = pack_bf16x2(p0, p1);
             pk[16 + c / 2] = pack_bf16x2(p2, p3);
           }
