@@ -46,6 +46,9 @@ DESCR = {
 }
 
 
+METRIC = "verified tree tokens/s (whole verify step: prepare + tree attention + acceptance + commit)"
+
+
 def attn_algorithmic_bytes(inp) -> int:
     """Bytes a tree_verify_attn launch must move at minimum: prefix K+V once per (sequence, KV
     head), tree K+V, Q read and O written."""
@@ -354,7 +357,7 @@ def run_ours(args, rank, world, local_rank):
                      "tensor_frac": round(flops / (attn_ms * 1e-3) / 1e12 / tpeak, 4)})
         value = aggregate_rate(tok, world, args.steps, step_ms)
         res = {
-            "metric": "verified tree tokens/s (whole verify step: prepare + tree attention + acceptance + commit)",
+            "metric": METRIC,
             "value": round(value, 1),
             "unit": "tokens/s",
             "n_gpus": world,
@@ -448,11 +451,13 @@ def run_reference(args, rank):
     step_tokens = tokens_per_step(inp)
     cb = {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
           "sample": f"per step: {desc}; {args.steps} steps, {secs:.1f} s"}
-    return {"impl": "reference", "metric": "verified tree tokens/s (whole verify step)", "value": round(value, 2),
-            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2),
+            "unit": "tokens/s", "n_gpus": args.gpus, "ran_on": "one host core of rank 0 (the fp64 oracle)",
+            "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(step_tokens / value * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; workloads module)",
-            "config": {"workload": f"{args.workload}: {DESCR[args.workload]}"}, "cpu_baseline": cb,
+            "config": {"workload": f"{args.workload}: {DESCR[args.workload]}", "tokens_per_step_per_gpu": step_tokens},
+            "cpu_baseline": cb,
             "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
