@@ -288,3 +288,6 @@ def verify_step(inp: dict, rows=None):
         acc = chain_sample(inp["z_p"], inp["z_q"], inp["x"], inp["u"], inp["T"])
         res = kv_commit(inp, acc["accept_len"], None, "length")
     return out, acc, res
+
+
+from .draft_tree import DraftTree, draft_tree_build  # noqa: E402,F401
