@@ -327,6 +327,51 @@ tsd_status tsd_tree_accept_commit(const void *logits, tsd_dtype logits_dtype, in
                                   int32_t *path, int32_t *out_tokens, void *workspace, size_t ws_bytes,
                                   int32_t *status, void *stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Device-side draft tree build (EAGLE-2 style): tsd_draft_tree_init / _expand / _finalize
+ * ([SO] "EAGLE": EAGLE-2 shapes the tree dynamically from the Top-K candidates of every node
+ * and scores the draft sequences).  Reading of that passage: a node's children are its K most
+ * likely draft tokens (ties -> lower token id), a node's score is the cumulative draft
+ * log-probability of its root->node path, the next nodes to expand are the F best children
+ * (score desc, then node index), and the final tree keeps the root plus the keep-1 best nodes
+ * (same order), renumbered by (depth, score desc, node index) with parents remapped -- the
+ * parent[] / tokens the verify step takes.  The tree lives on the device between draft steps.
+ *
+ * tsd_draft_tree holds caller-owned device arrays:
+ *   parent, token, depth [B, max_nodes] int32; score [B, max_nodes] fp64;
+ *   num_nodes [B]; frontier [B, F] (node ids, best first); num_frontier [B];
+ *   F <= 16 frontier width.
+ * init: node 0 = root (token root_token[b], score 0), frontier = [0]; status[b] = 0.
+ * expand: draft_logits [B, F, V] (row f = the draft distribution after frontier node f; rows
+ *   past num_frontier[b] are ignored), K <= min(16, V) children per node, V <= 64 * 16384; appends
+ *   num_frontier * K nodes (in frontier order, then rank order) and replaces the frontier.
+ *   Scores: fp32 exponentials summed in fp64, log-sum-exp and scores in fp64.  Capacity
+ *   overflow flags TSD_ERR_CAPACITY in status[b] and leaves the tree unchanged.
+ *   workspace >= tsd_draft_tree_expand_workspace_size(B, F, K, V) bytes.  Two launches.
+ * finalize: parent_out [B, keep] int32 (root -1, padding -1), tokens_out [B, keep] (padding 0),
+ *   num_nodes_out [B] = min(keep, nodes); max_nodes <= 4096.  One launch.
+ * A flagged sequence (status[b] != 0) is skipped by expand and finalised empty.
+ * --------------------------------------------------------------------------------------- */
+typedef struct tsd_draft_tree {
+  int32_t *parent;
+  int32_t *token;
+  double *score;
+  int32_t *depth;
+  int32_t *num_nodes;
+  int32_t *frontier;
+  int32_t *num_frontier;
+  int max_nodes;
+  int F;
+} tsd_draft_tree;
+
+tsd_status tsd_draft_tree_init(const tsd_draft_tree *tree, const int32_t *root_token, int B, int32_t *status,
+                               void *stream);
+size_t tsd_draft_tree_expand_workspace_size(int B, int F, int K, int V);
+tsd_status tsd_draft_tree_expand(const tsd_draft_tree *tree, const void *draft_logits, tsd_dtype dtype, int V, int K,
+                                 int B, void *workspace, size_t ws_bytes, int32_t *status, void *stream);
+tsd_status tsd_draft_tree_finalize(const tsd_draft_tree *tree, int B, int keep, int32_t *parent_out,
+                                   int32_t *tokens_out, int32_t *num_nodes_out, int32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -43,9 +43,9 @@ def logsumexp(z: np.ndarray) -> float:
 
 
 def top_k_tokens(z: np.ndarray, K: int) -> list:
-    """The K largest entries of z, ties -> lower index, best first."""
-    order = sorted(range(len(z)), key=lambda v: (-z[v], v))
-    return order[:K]
+    """The K largest entries of z, ties -> lower index, best first (a stable sort of -z)."""
+    order = np.lexsort((np.arange(len(z)), -z))
+    return [int(v) for v in order[:K]]
 
 
 class DraftTree:
@@ -71,20 +71,28 @@ class DraftTree:
                 children.append(len(self.parent) - 1)
         ranked = sorted(children, key=lambda i: (-self.score[i], i))
         if len(ranked) > F:
-            self.margins.append(self.score[ranked[F - 1]] - self.score[ranked[F]])
+            self.margins.append(self._gap(ranked[F - 1], ranked[F]))
         self.frontier = ranked[:F]
+
+    def _gap(self, a: int, b: int) -> float:
+        """Score gap of a decision between nodes a and b.  Siblings with equal scores (the same
+        draft logit under the same parent) tie exactly on any arithmetic and are ordered by
+        index alike everywhere, so they decide nothing; any other gap is the decision margin."""
+        if self.parent[a] == self.parent[b] and self.score[a] == self.score[b]:
+            return np.inf
+        return abs(self.score[a] - self.score[b])
 
     def finalize(self, keep: int):
         """Returns (parent int32[n], tokens int32[n]) of the kept tree, n = min(keep, nodes)."""
         cand = sorted(range(1, len(self.parent)), key=lambda i: (-self.score[i], i))
         if len(cand) > keep - 1 and keep >= 2:
-            self.margins.append(self.score[cand[keep - 2]] - self.score[cand[keep - 1]])
+            self.margins.append(self._gap(cand[keep - 2], cand[keep - 1]))
         chosen = cand[: max(keep - 1, 0)]
         kept = [0] + sorted(chosen, key=lambda i: (self.depth[i], -self.score[i], i))
         # order decisions inside one depth also rest on score comparisons
         for a, b in zip(kept[1:], kept[2:]):
             if self.depth[a] == self.depth[b]:
-                self.margins.append(self.score[a] - self.score[b])
+                self.margins.append(self._gap(a, b))
         remap = {old: new for new, old in enumerate(kept)}
         parent = np.array([-1 if self.parent[o] < 0 else remap[self.parent[o]] for o in kept], np.int32)
         tokens = np.array([self.token[o] for o in kept], np.int32)

@@ -58,6 +58,17 @@ class KVCacheDesc(C.Structure):
                 ("block_size", _I), ("num_blocks", _I)]
 
 
+class DraftTreeDesc(C.Structure):
+    """tsd_draft_tree: the device arrays of a draft tree under construction."""
+    _fields_ = [("parent", _P), ("token", _P), ("score", _P), ("depth", _P), ("num_nodes", _P), ("frontier", _P),
+                ("num_frontier", _P), ("max_nodes", _I), ("F", _I)]
+
+
+_DT = C.POINTER(DraftTreeDesc)
+_SIGS["tsd_draft_tree_init"] = (_I, [_DT, _P, _I, _P, _P])
+_SIGS["tsd_draft_tree_expand_workspace_size"] = (_SZ, [_I, _I, _I, _I])
+_SIGS["tsd_draft_tree_expand"] = (_I, [_DT, _P, _I, _I, _I, _I, _P, _SZ, _P, _P])
+_SIGS["tsd_draft_tree_finalize"] = (_I, [_DT, _I, _I, _P, _P, _P, _P, _P])
 _SIGS["tsd_tree_accept_commit"] = (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, C.POINTER(KVCacheDesc), _P, _P, _I,
                                         _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P, _P])
 
@@ -343,6 +354,57 @@ def tree_accept_commit(logits, tokens, parent_s, k_cache, v_cache, prefix_len, k
                                       _ptr(status), _stream(stream))
     _check(rc, "tsd_tree_accept_commit")
     return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
+
+
+# ----------------------------------------------------------------------------- draft tree
+class DraftTree:
+    """A batch of EAGLE-2 draft trees built on the device (tsd_draft_tree_*).
+
+    ``init(root_tokens)`` starts every tree at its root; ``expand(draft_logits, K)`` takes the
+    [B, F, V] draft logits of the current frontier nodes (row f after frontier node f) and adds
+    their top-K children; ``finalize(keep)`` returns the parent[] / tokens / num_nodes of the
+    kept tree, ready for ``tree_prepare`` and the verify step."""
+
+    def __init__(self, B: int, F: int, max_nodes: int, device="cuda"):
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.B, self.F, self.max_nodes = B, F, max_nodes
+        self.parent = torch.zeros(B, max_nodes, **i32)
+        self.token = torch.zeros(B, max_nodes, **i32)
+        self.score = torch.zeros(B, max_nodes, dtype=torch.float64, device=dev)
+        self.depth = torch.zeros(B, max_nodes, **i32)
+        self.num_nodes = torch.zeros(B, **i32)
+        self.frontier = torch.zeros(B, F, **i32)
+        self.num_frontier = torch.zeros(B, **i32)
+        self.status = torch.zeros(B, **i32)
+        self._ws = None
+        self.desc = DraftTreeDesc(_ptr(self.parent), _ptr(self.token), _ptr(self.score), _ptr(self.depth),
+                                  _ptr(self.num_nodes), _ptr(self.frontier), _ptr(self.num_frontier), max_nodes, F)
+
+    def init(self, root_tokens, stream=None):
+        _check(lib().tsd_draft_tree_init(C.byref(self.desc), _i32(root_tokens, "root_tokens"), self.B,
+                                         _ptr(self.status), _stream(stream)), "tsd_draft_tree_init")
+
+    def expand(self, draft_logits, K: int, stream=None):
+        B, F, V = draft_logits.shape
+        if B != self.B or F != self.F:
+            raise TsdError("draft_logits must be [B, F, V] of this tree")
+        nbytes = int(lib().tsd_draft_tree_expand_workspace_size(B, F, K, V))
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=draft_logits.device)
+        _check(lib().tsd_draft_tree_expand(C.byref(self.desc), _ptr(draft_logits), _dt(draft_logits), V, K, B,
+                                           _ptr(self._ws), nbytes, _ptr(self.status), _stream(stream)),
+               "tsd_draft_tree_expand")
+
+    def finalize(self, keep: int, parent=None, tokens=None, num_nodes=None, stream=None):
+        dev = self.parent.device
+        parent = torch.empty(self.B, keep, dtype=torch.int32, device=dev) if parent is None else parent
+        tokens = torch.empty(self.B, keep, dtype=torch.int32, device=dev) if tokens is None else tokens
+        num_nodes = torch.empty(self.B, dtype=torch.int32, device=dev) if num_nodes is None else num_nodes
+        _check(lib().tsd_draft_tree_finalize(C.byref(self.desc), self.B, keep, _ptr(parent), _ptr(tokens),
+                                             _ptr(num_nodes), _ptr(self.status), _stream(stream)),
+               "tsd_draft_tree_finalize")
+        return {"parent": parent, "tokens": tokens, "num_nodes": num_nodes}
 
 
 from .step import VerifyStep  # noqa: E402,F401

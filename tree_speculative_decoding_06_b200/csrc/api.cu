@@ -275,4 +275,52 @@ tsd_status tsd_tree_accept_commit(const void* logits, tsd_dtype logits_dtype, in
                               workspace, S(stream));
 }
 
+static bool draft_args(const tsd_draft_tree* tree, int B, DraftTreeArgs& t) {
+  if (!tree || B < 0 || B > 65535 || tree->max_nodes < 1 || tree->F < 1 || tree->F > 16) return false;
+  if (B > 0 && (!tree->parent || !tree->token || !tree->score || !tree->depth || !tree->num_nodes ||
+                !tree->frontier || !tree->num_frontier))
+    return false;
+  t.parent = tree->parent, t.token = tree->token, t.score = tree->score, t.depth = tree->depth;
+  t.num_nodes = tree->num_nodes, t.frontier = tree->frontier, t.num_frontier = tree->num_frontier;
+  t.max_nodes = tree->max_nodes, t.F = tree->F, t.B = B;
+  return true;
+}
+
+tsd_status tsd_draft_tree_init(const tsd_draft_tree* tree, const int32_t* root_token, int B, int32_t* status,
+                               void* stream) {
+  DraftTreeArgs t{};
+  if (!draft_args(tree, B, t)) return TSD_ERR_INVALID_ARG;
+  if (B == 0) return TSD_OK;
+  if (!root_token || !status) return TSD_ERR_INVALID_ARG;
+  return launch_draft_init(t, root_token, status, S(stream));
+}
+
+size_t tsd_draft_tree_expand_workspace_size(int B, int F, int K, int V) {
+  if (B <= 0 || F <= 0 || K <= 0 || V <= 0) return 0;
+  return draft_expand_ws(B, F, K, V);
+}
+
+tsd_status tsd_draft_tree_expand(const tsd_draft_tree* tree, const void* draft_logits, tsd_dtype dtype, int V, int K,
+                                 int B, void* workspace, size_t ws_bytes, int32_t* status, void* stream) {
+  if (!dtype_ok(dtype)) return TSD_ERR_UNSUPPORTED_DTYPE;
+  DraftTreeArgs t{};
+  if (!draft_args(tree, B, t)) return TSD_ERR_INVALID_ARG;
+  if (V <= 0 || V > 64 * 16384 || K < 1 || K > 16 || K > V) return TSD_ERR_INVALID_ARG;
+  if (B == 0) return TSD_OK;
+  if (!draft_logits || !status) return TSD_ERR_INVALID_ARG;
+  const size_t need = draft_expand_ws(B, t.F, K, V);
+  if (workspace == nullptr || ws_bytes < need) return TSD_ERR_WORKSPACE;
+  return launch_draft_expand(t, draft_logits, dtype, V, K, workspace, status, S(stream));
+}
+
+tsd_status tsd_draft_tree_finalize(const tsd_draft_tree* tree, int B, int keep, int32_t* parent_out,
+                                   int32_t* tokens_out, int32_t* num_nodes_out, int32_t* status, void* stream) {
+  DraftTreeArgs t{};
+  if (!draft_args(tree, B, t)) return TSD_ERR_INVALID_ARG;
+  if (keep < 1 || tree->max_nodes > 4096) return TSD_ERR_INVALID_ARG;
+  if (B == 0) return TSD_OK;
+  if (!parent_out || !tokens_out || !num_nodes_out || !status) return TSD_ERR_INVALID_ARG;
+  return launch_draft_finalize(t, keep, parent_out, tokens_out, num_nodes_out, status, S(stream));
+}
+
 }  // extern "C"

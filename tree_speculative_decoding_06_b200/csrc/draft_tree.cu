@@ -1,0 +1,362 @@
+// tsd_draft_tree_init / _expand / _finalize: the EAGLE-2 draft tree built on the device.
+//
+// "Acelerando Sonar a traves de la especulacion", section "EAGLE": EAGLE-2 shapes the draft tree
+// dynamically, expanding the Top-K candidates of every node and scoring the draft sequences.
+// Reading of that passage (the pages give no more): a node's children are its K most likely
+// draft tokens, a node's score is the cumulative draft log-probability of its root->node path,
+// the next nodes to expand are the F best children, and the final tree keeps the root and the
+// best keep-1 nodes by score, ordered by (depth, score desc, node index).
+//
+// Expansion is two launches: a vocabulary scan (one CTA per 16384-token chunk of every frontier
+// row: chunk maximum, fp64 sum of fp32 exponentials, chunk top-K) and one CTA per sequence that
+// merges the chunks (log-sum-exp, row top-K), appends the children and picks the new frontier by
+// rank counting.  Finalisation is one CTA per sequence: rank every node by score, keep the best,
+// renumber by (depth, score, index), remap parents.  Scores are fp64.
+#include <climits>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tsd {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kChunk = 16384;           // vocabulary entries per scan CTA
+constexpr int kMaxK = 16;               // children per node
+constexpr int kMaxFinalNodes = 4096;    // tree capacity finalize stages on chip
+
+__host__ __device__ inline int dt_chunks(int V) { return (V + kChunk - 1) / kChunk; }
+// per (sequence, frontier row, chunk): fp64 sum, fp32 max, then K (value, index) pairs
+__host__ __device__ inline size_t dt_rec_bytes(int K) { return ((size_t)16 + (size_t)8 * K + 15) & ~(size_t)15; }
+
+struct ChunkRec {
+  double s;
+  float m;
+  float pad;
+};
+
+__device__ __forceinline__ bool better_node(double sa, int ia, double sb, int ib) {
+  return sa > sb || (sa == sb && ia < ib);
+}
+
+// Insert (x, v) into the sorted (best first) list (tv, ti) of length K <= kMaxK: the new entry
+// bubbles in, the last one falls out.  Static indices only (the list stays in registers).
+__device__ __forceinline__ void topk_insert(float (&tv)[kMaxK], int (&ti)[kMaxK], int K, float x, int v) {
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) {
+    if (k < K && better(x, v, tv[k], ti[k])) {
+      const float t = tv[k];
+      const int u = ti[k];
+      tv[k] = x, ti[k] = v;
+      x = t, v = u;
+    }
+  }
+}
+__device__ __forceinline__ void topk_at(const float (&tv)[kMaxK], const int (&ti)[kMaxK], int k, float& x, int& v) {
+  x = -INFINITY, v = INT_MAX;
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j)
+    if (j == k) x = tv[j], v = ti[j];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict__ logits, int V, int F, int K,
+                                                            int chunks, uint8_t* __restrict__ ws) {
+  pdl_trigger();
+  const int c = blockIdx.x, f = blockIdx.y, b = blockIdx.z;
+  const T* row = logits + ((size_t)b * F + f) * V;
+  const int lo = c * kChunk, hi = min(V, lo + kChunk);
+  float tv[kMaxK];
+  int ti[kMaxK];
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) tv[k] = -INFINITY, ti[k] = INT_MAX;
+  float thr_v = -INFINITY;   // the K-th best so far
+  int thr_i = INT_MAX;
+  float m = -INFINITY;
+  auto take = [&](float x, int v) {
+    m = fmaxf(m, x);
+    if (better(x, v, thr_v, thr_i)) {
+      topk_insert(tv, ti, K, x, v);
+      topk_at(tv, ti, K - 1, thr_v, thr_i);
+    }
+  };
+  if ((V & 7) == 0) {
+    for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
+      float x[8];
+      load8<T>(row, v, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) take(x[e], v + e);
+    }
+  } else {
+    for (int v = lo + threadIdx.x; v < hi; v += kThreads) take(load1(row, v), v);
+  }
+  // chunk maximum
+  __shared__ float s_m[kThreads / 32];
+  __shared__ double s_s[kThreads / 32];
+  __shared__ float s_bv[kThreads / 32];
+  __shared__ int s_bi[kThreads / 32], s_bt[kThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float wm = warp_max(m);
+  if (lane == 0) s_m[warp] = wm;
+  __syncthreads();
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) M = fmaxf(M, s_m[w]);
+  // fp64 sum of fp32 exponentials relative to the chunk maximum (second pass, cache-resident)
+  double sum = 0.0;
+  if (M != -INFINITY) {
+    if ((V & 7) == 0) {
+      for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
+        float x[8];
+        load8<T>(row, v, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sum += (double)expf(x[e] - M);
+      }
+    } else {
+      for (int v = lo + threadIdx.x; v < hi; v += kThreads) sum += (double)expf(load1(row, v) - M);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) s_s[warp] = sum;
+  // chunk top-K: K rounds of a block argmax over every thread's current head
+  __shared__ float s_topv[kMaxK];
+  __shared__ int s_topi[kMaxK];
+  int h = 0;
+  for (int r = 0; r < K; ++r) {
+    float hv;
+    int hi_;
+    if (h < K) topk_at(tv, ti, h, hv, hi_);
+    else hv = -INFINITY, hi_ = INT_MAX;
+    float bv = hv;
+    int bi = hi_, bt = threadIdx.x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const int ot = __shfl_xor_sync(0xffffffffu, bt, o);
+      if (better(ov, oi, bv, bi)) bv = ov, bi = oi, bt = ot;
+    }
+    __syncthreads();   // s_bv of the previous round has been read
+    if (lane == 0) s_bv[warp] = bv, s_bi[warp] = bi, s_bt[warp] = bt;
+    __syncthreads();
+    float gv = -INFINITY;
+    int gi = INT_MAX, gt = -1;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w)
+      if (better(s_bv[w], s_bi[w], gv, gi)) gv = s_bv[w], gi = s_bi[w], gt = s_bt[w];
+    if (threadIdx.x == gt) ++h;
+    if (threadIdx.x == 0) s_topv[r] = gv, s_topi[r] = gi;
+  }
+  __syncthreads();
+  pdl_wait();   // the previous expansion may still be reading the workspace
+  if (threadIdx.x == 0) {
+    double S = 0.0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) S += s_s[w];
+    uint8_t* rec = ws + (((size_t)b * F + f) * chunks + c) * dt_rec_bytes(K);
+    ChunkRec cr;
+    cr.s = S, cr.m = M, cr.pad = 0.f;
+    *reinterpret_cast<ChunkRec*>(rec) = cr;
+    float* vals = reinterpret_cast<float*>(rec + 16);
+    int* idxs = reinterpret_cast<int*>(rec + 16 + 4 * K);
+    for (int k = 0; k < K; ++k) vals[k] = s_topv[k], idxs[k] = s_topi[k];
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) draft_init_kernel(DraftTreeArgs t, const int32_t* __restrict__ root_token,
+                                                              int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= t.B) return;
+  const size_t base = (size_t)b * t.max_nodes;
+  t.parent[base] = -1;
+  t.token[base] = root_token[b];
+  t.score[base] = 0.0;
+  t.depth[base] = 0;
+  t.num_nodes[b] = 1;
+  t.frontier[(size_t)b * t.F] = 0;
+  t.num_frontier[b] = 1;
+  status[b] = 0;
+}
+
+__global__ void __launch_bounds__(kThreads) draft_expand_kernel(DraftTreeArgs t, int K, int chunks,
+                                                                const uint8_t* __restrict__ ws,
+                                                                int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ double s_sc[kMaxK * kMaxK];
+  __shared__ int s_id[kMaxK * kMaxK];
+  const int b = blockIdx.x;
+  const int nf = t.num_frontier[b], n0 = t.num_nodes[b];
+  const size_t base = (size_t)b * t.max_nodes;
+  if (status[b] != 0 || nf <= 0) return;
+  if (nf > t.F || (long long)n0 + (long long)nf * K > t.max_nodes) {
+    if (threadIdx.x == 0) flag_status(status, b, TSD_ERR_CAPACITY);
+    return;
+  }
+  // one thread per frontier row: merge the chunk records, append the row's K children
+  const int f = threadIdx.x;
+  if (f < nf) {
+    const size_t rb = dt_rec_bytes(K);
+    const uint8_t* recs = ws + ((size_t)b * t.F + f) * chunks * rb;
+    float M = -INFINITY;
+    for (int c = 0; c < chunks; ++c) M = fmaxf(M, reinterpret_cast<const ChunkRec*>(recs + c * rb)->m);
+    double S = 0.0;
+    for (int c = 0; c < chunks; ++c) {
+      const ChunkRec* cr = reinterpret_cast<const ChunkRec*>(recs + c * rb);
+      if (cr->m != -INFINITY) S += cr->s * exp((double)cr->m - (double)M);
+    }
+    const double lse = (double)M + log(S);
+    const int p = t.frontier[(size_t)b * t.F + f];
+    const double sp = t.score[base + p];
+    const int dp = t.depth[base + p];
+    int head[64];   // per-chunk read position of the K-way merge (chunks <= 64)
+    for (int c = 0; c < chunks; ++c) head[c] = 0;
+    for (int k = 0; k < K; ++k) {
+      float bv = -INFINITY;
+      int bi = INT_MAX, bc = -1;
+      for (int c = 0; c < chunks; ++c) {
+        if (head[c] >= K) continue;
+        const uint8_t* rec = recs + c * rb;
+        const float v = reinterpret_cast<const float*>(rec + 16)[head[c]];
+        const int i = reinterpret_cast<const int*>(rec + 16 + 4 * K)[head[c]];
+        if (i != INT_MAX && better(v, i, bv, bi)) bv = v, bi = i, bc = c;
+      }
+      if (bc >= 0) ++head[bc];
+      const int node = n0 + f * K + k;
+      const double sc = sp + ((double)bv - lse);
+      t.parent[base + node] = p;
+      t.token[base + node] = bi == INT_MAX ? 0 : bi;
+      t.score[base + node] = sc;
+      t.depth[base + node] = dp + 1;
+      s_sc[f * K + k] = sc;
+      s_id[f * K + k] = node;
+    }
+  }
+  __syncthreads();
+  // new frontier: rank of every child among all children by (score desc, node index asc)
+  const int nc = nf * K;
+  for (int j = threadIdx.x; j < nc; j += blockDim.x) {
+    int rank = 0;
+    for (int i = 0; i < nc; ++i) rank += better_node(s_sc[i], s_id[i], s_sc[j], s_id[j]) ? 1 : 0;
+    if (rank < t.F) t.frontier[(size_t)b * t.F + rank] = s_id[j];
+  }
+  if (threadIdx.x == 0) {
+    t.num_nodes[b] = n0 + nc;
+    t.num_frontier[b] = nc < t.F ? nc : t.F;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) draft_finalize_kernel(DraftTreeArgs t, int keep,
+                                                                  int32_t* __restrict__ parent_out,
+                                                                  int32_t* __restrict__ tokens_out,
+                                                                  int32_t* __restrict__ num_out,
+                                                                  int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int b = blockIdx.x;
+  const int n = t.num_nodes[b];
+  const size_t base = (size_t)b * t.max_nodes;
+  int32_t* prow = parent_out + (size_t)b * keep;
+  int32_t* trow = tokens_out + (size_t)b * keep;
+  const bool bad = status[b] != 0 || n < 1 || n > t.max_nodes;
+  const int kept_n = bad ? 0 : min(keep, n);
+  if (bad) {
+    for (int i = threadIdx.x; i < keep; i += blockDim.x) prow[i] = -1, trow[i] = 0;
+    if (threadIdx.x == 0) num_out[b] = 0;
+    return;
+  }
+  double* s_sc = reinterpret_cast<double*>(smem);
+  int* s_dep = reinterpret_cast<int*>(s_sc + n);
+  int* s_map = s_dep + n;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    s_sc[i] = t.score[base + i];
+    s_dep[i] = t.depth[base + i];
+    s_map[i] = -1;
+  }
+  __syncthreads();
+  // kept: the root and the kept_n - 1 best other nodes by (score desc, index asc)
+  for (int i = 1 + threadIdx.x; i < n; i += blockDim.x) {
+    int rank = 0;
+    for (int j = 1; j < n; ++j) rank += better_node(s_sc[j], j, s_sc[i], i) ? 1 : 0;
+    if (rank < kept_n - 1) s_map[i] = -2;   // kept, position below
+  }
+  __syncthreads();
+  // position among the kept by (depth asc, score desc, index asc); the root is position 0
+  for (int i = 1 + threadIdx.x; i < n; i += blockDim.x) {
+    if (s_map[i] != -2) continue;
+    int pos = 1;
+    for (int j = 1; j < n; ++j) {
+      if (j == i) continue;
+      const int mj = s_map[j];
+      if (mj == -1) continue;   // not kept (a kept node's entry is -2 or already its position)
+      const bool before = s_dep[j] < s_dep[i] || (s_dep[j] == s_dep[i] && better_node(s_sc[j], j, s_sc[i], i));
+      pos += before ? 1 : 0;
+    }
+    s_map[i] = -1000 - pos;     // kept marker that stays distinct from -1 while others still read
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    if (s_map[i] <= -1000) s_map[i] = -1000 - s_map[i];
+  if (threadIdx.x == 0) s_map[0] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int pos = s_map[i];
+    if (pos < 0) continue;
+    const int p = t.parent[base + i];
+    int np = -1;
+    if (i > 0) {
+      np = (p >= 0 && p < n) ? s_map[p] : -1;
+      if (np < 0) flag_status(status, b, TSD_ERR_BAD_TREE, i);   // not ancestor-closed (never for scores)
+    }
+    prow[pos] = np;
+    trow[pos] = t.token[base + i];
+  }
+  for (int i = kept_n + threadIdx.x; i < keep; i += blockDim.x) prow[i] = -1, trow[i] = 0;
+  if (threadIdx.x == 0) num_out[b] = kept_n;
+}
+
+}  // namespace
+
+size_t draft_expand_ws(int B, int F, int K, int V) { return (size_t)B * F * dt_chunks(V) * dt_rec_bytes(K); }
+
+tsd_status launch_draft_init(const DraftTreeArgs& t, const int32_t* root_token, int32_t* status, cudaStream_t stream) {
+  if (t.B == 0) return TSD_OK;
+  launch_pdl(draft_init_kernel, dim3((t.B + kThreads - 1) / kThreads), dim3(kThreads), 0, stream, t, root_token, status);
+  return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+}
+
+tsd_status launch_draft_expand(const DraftTreeArgs& t, const void* logits, tsd_dtype dtype, int V, int K, void* ws,
+                               int32_t* status, cudaStream_t stream) {
+  if (t.B == 0) return TSD_OK;
+  if (K < 1 || K > kMaxK || t.F < 1 || t.F > kMaxK || dt_chunks(V) > 64) return TSD_ERR_INVALID_ARG;
+  const int chunks = dt_chunks(V);
+  dim3 grid(chunks, t.F, t.B);
+  if (dtype == TSD_BF16)
+    launch_pdl(draft_row_stats<__nv_bfloat16>, grid, dim3(kThreads), 0, stream,
+               reinterpret_cast<const __nv_bfloat16*>(logits), V, t.F, K, chunks, reinterpret_cast<uint8_t*>(ws));
+  else
+    launch_pdl(draft_row_stats<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(logits), V, t.F,
+               K, chunks, reinterpret_cast<uint8_t*>(ws));
+  if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
+  launch_pdl(draft_expand_kernel, dim3(t.B), dim3(kThreads), 0, stream, t, K, chunks, (const uint8_t*)ws, status);
+  return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+}
+
+tsd_status launch_draft_finalize(const DraftTreeArgs& t, int keep, int32_t* parent_out, int32_t* tokens_out,
+                                 int32_t* num_out, int32_t* status, cudaStream_t stream) {
+  if (t.B == 0) return TSD_OK;
+  if (t.max_nodes > kMaxFinalNodes || keep < 1) return TSD_ERR_INVALID_ARG;
+  const size_t smem = (size_t)t.max_nodes * (8 + 4 + 4);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(draft_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  launch_pdl(draft_finalize_kernel, dim3(t.B), dim3(kThreads), smem, stream, t, keep, parent_out, tokens_out, num_out,
+             status);
+  return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+}
+
+}  // namespace tsd
