@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kThreads) draft_expand_kernel(DraftTreeArgs t,
                                                                 int32_t* __restrict__ status) {
   pdl_trigger();
   pdl_wait();
+  extern __shared__ __align__(16) uint8_t s_recs[];
   __shared__ double s_sc[kMaxK * kMaxK];
   __shared__ int s_id[kMaxK * kMaxK];
   const int b = blockIdx.x;
@@ -197,11 +198,20 @@ __global__ void __launch_bounds__(kThreads) draft_expand_kernel(DraftTreeArgs t,
     if (threadIdx.x == 0) flag_status(status, b, TSD_ERR_CAPACITY);
     return;
   }
+  // every chunk record of the sequence into shared memory with one coalesced read, so the row
+  // merges below do not chain dependent global loads
+  const size_t rb = dt_rec_bytes(K);
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(ws + (size_t)b * t.F * chunks * rb);
+    uint4* dst = reinterpret_cast<uint4*>(s_recs);
+    const int n16 = (int)((size_t)nf * chunks * rb / 16);
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = src[i];
+  }
+  __syncthreads();
   // one thread per frontier row: merge the chunk records, append the row's K children
   const int f = threadIdx.x;
   if (f < nf) {
-    const size_t rb = dt_rec_bytes(K);
-    const uint8_t* recs = ws + ((size_t)b * t.F + f) * chunks * rb;
+    const uint8_t* recs = s_recs + (size_t)f * chunks * rb;
     float M = -INFINITY;
     for (int c = 0; c < chunks; ++c) M = fmaxf(M, reinterpret_cast<const ChunkRec*>(recs + c * rb)->m);
     double S = 0.0;
@@ -343,7 +353,10 @@ tsd_status launch_draft_expand(const DraftTreeArgs& t, const void* logits, tsd_d
     launch_pdl(draft_row_stats<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(logits), V, t.F,
                K, chunks, reinterpret_cast<uint8_t*>(ws));
   if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
-  launch_pdl(draft_expand_kernel, dim3(t.B), dim3(kThreads), 0, stream, t, K, chunks, (const uint8_t*)ws, status);
+  const size_t smem = (size_t)t.F * chunks * dt_rec_bytes(K);   // <= 16 x 64 x 144 B
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(draft_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  launch_pdl(draft_expand_kernel, dim3(t.B), dim3(kThreads), smem, stream, t, K, chunks, (const uint8_t*)ws, status);
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }
 
