@@ -68,3 +68,31 @@ def test_workspace_sizes_are_consistent():
     assert a == b
     assert tsd.tree_accept_greedy_workspace_size(8, 512, 128256) == 8 * 512 * 16 * 8
     assert tsd.chain_accept_sample_workspace_size(64, 5, 128256) > 64 * 11 * 16 * 8
+
+
+def test_host_checks_of_the_fused_and_draft_tree_entry_points():
+    L = tsd.lib()
+    cache = tsd.KVCacheDesc(None, None, None, 16, None, 0, 0, 0)
+    # fused acceptance + commit: a null cache struct, an empty batch, a missing pointer
+    assert L.tsd_tree_accept_commit(None, 1, 16, None, None, None, None, 1, 4, 3, None, None, None, 2, 64, 1, 0,
+                                    None, 0, None, None, None, None, None, 0, None, None) == 1
+    assert L.tsd_tree_accept_commit(None, 1, 16, None, None, None, None, 0, 4, 3, ctypes.byref(cache), None, None, 2,
+                                    64, 1, 0, None, 0, None, None, None, None, None, 0, None, None) == 0
+    assert L.tsd_tree_accept_commit(None, 1, 16, None, None, None, None, 1, 4, 3, ctypes.byref(cache), None, None, 2,
+                                    64, 1, 0, None, 0, None, None, None, None, None, 0, None, None) == 1
+    assert L.tsd_tree_accept_commit(None, 7, 16, None, None, None, None, 1, 4, 3, ctypes.byref(cache), None, None, 2,
+                                    64, 1, 0, None, 0, None, None, None, None, None, 0, None, None) == 2
+    # draft tree: frontier width and K limits, K above V, empty batches, workspace
+    d = tsd.DraftTreeDesc(None, None, None, None, None, None, None, 64, 4)
+    assert L.tsd_draft_tree_init(ctypes.byref(d), None, 0, None, None) == 0
+    assert L.tsd_draft_tree_init(ctypes.byref(d), None, 1, None, None) == 1          # null arrays
+    wide = tsd.DraftTreeDesc(None, None, None, None, None, None, None, 64, 17)
+    assert L.tsd_draft_tree_init(ctypes.byref(wide), None, 0, None, None) == 1       # F > 16
+    assert L.tsd_draft_tree_expand(ctypes.byref(d), None, 1, 100, 17, 0, None, 0, None, None) == 1   # K > 16
+    assert L.tsd_draft_tree_expand(ctypes.byref(d), None, 1, 8, 10, 0, None, 0, None, None) == 1     # K > V
+    assert L.tsd_draft_tree_expand(ctypes.byref(d), None, 9, 100, 4, 0, None, 0, None, None) == 2    # dtype
+    assert L.tsd_draft_tree_finalize(ctypes.byref(d), 0, 0, None, None, None, None, None) == 1        # keep 0
+    big = tsd.DraftTreeDesc(None, None, None, None, None, None, None, 5000, 4)
+    assert L.tsd_draft_tree_finalize(ctypes.byref(big), 0, 8, None, None, None, None, None) == 1      # > 4096 nodes
+    # one record of (2 x 4 + 16) bytes rounded to 16, per (sequence, row, 16384-token chunk)
+    assert tsd.lib().tsd_draft_tree_expand_workspace_size(2, 10, 10, 128256) == 2 * 10 * 8 * 96
