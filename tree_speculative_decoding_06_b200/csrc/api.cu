@@ -2,6 +2,7 @@
 // caller's stream.  No allocation, no synchronisation, no state kept between calls.
 #include <cstdio>
 
+#include "draft_tree.h"
 #include "kernels.h"
 #include "tsd.h"
 

@@ -15,6 +15,7 @@
 #include <climits>
 
 #include "common.cuh"
+#include "draft_tree.h"
 #include "kernels.h"
 
 namespace tsd {
