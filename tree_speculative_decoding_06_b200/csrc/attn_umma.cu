@@ -4,26 +4,33 @@
 // summary sec. 2: a tree token attends to the committed prefix and to its own ancestors only;
 // "Acelerando Sonar a traves de la especulacion", section "EAGLE": the mask touches only the
 // tree's keys), built for Blackwell:
-//   * a CTA owns 128 query rows (G heads x 128/G tree nodes of one KV head) and a range of 64-key
-//     tiles of one sequence; every K/V tile is read from memory once per 128 rows;
+//   * a CTA owns 128 query rows (G heads x 128/G tree nodes of one KV head), or two such tiles
+//     when a KV head has more than 128 rows, and a range of 64-key tiles of one sequence; every
+//     K/V tile is read from memory once per CTA;
 //   * two producer threads stream K and V tiles with TMA (128-byte swizzled boxes; paged caches
 //     box by block, the tree's K/V by node for one KV head) into separate rings: a K slot is
 //     released as soon as S = Q K^T has read it, a V slot after P V, so loads run several tiles
 //     ahead of the math;
-//   * one thread (warp 3) issues tcgen05.mma: S into one of four TMEM tiles (128 lanes x 64 fp32
-//     columns; two per softmax warpgroup, so the tensor cores compute a warpgroup's next S while
-//     it is still exponentiating the current one) and O += P V into one of two 128 x 128 fp32
-//     TMEM accumulators, with descriptors built once and advanced by constants;
+//   * warp 3 issues tcgen05.mma warp-collectively (one elected lane; descriptors built once and
+//     advanced by constants): S into TMEM tiles of 128 lanes x 64 fp32 columns (two per softmax
+//     warpgroup with one query tile, so the tensor cores compute a warpgroup's next S while it
+//     is still exponentiating the current one) and O += P V into two 128 x 128 fp32 TMEM
+//     accumulators;
 //   * P never touches shared memory: the softmax writes it as bf16 over the first half of its S
-//     tile in TMEM and the P V product reads its A operand from there, so shared-memory
-//     bandwidth is left to the TMA writes and the K and V operand reads;
-//   * two softmax warpgroups take alternate tiles (even / odd), each with its own two S tiles,
-//     O accumulator and running (max, sum) -- a split of the key range inside the CTA,
-//     merged by log-sum-exp in the epilogue.  In a warpgroup each warp owns one TMEM lane
-//     quarter, one query row per thread: a row's 64 scores come out of TMEM with one tcgen05.ld,
-//     so its max and sum need no shuffles.  The ancestor mask is applied only on tree tiles (bits
-//     rebuilt in shared memory at set-up); full prefix tiles take a lean path (no mask work).  The
-//     running max is raised lazily (only past a 2^8 growth), so O is rescaled in TMEM rarely.
+//     tile in TMEM and the P V product reads its A operand from there; with two query tiles the
+//     tiles themselves live in TMEM too (the A operand of S), so shared memory carries only the
+//     TMA writes and the K and V operand reads;
+//   * one query tile: two softmax warpgroups take alternate key tiles (even / odd), each with its
+//     own S tiles, O accumulator and running (max, sum) -- a split of the key range inside the
+//     CTA, merged by log-sum-exp in the epilogue; two query tiles: warpgroup w owns query tile w
+//     over every key tile.  In a warpgroup each warp owns one TMEM lane quarter, one query row
+//     per thread: a row's 64 scores come out of TMEM with one tcgen05.ld, so its max and sum need
+//     no shuffles.  The ancestor mask is applied only on tree tiles (bits built in shared memory
+//     by warp 1 from the staged parent slots while the first prefix tiles stream in); full
+//     prefix tiles take a lean path (no mask work, paired fp32 instructions).  The running max is
+//     raised lazily (only past a 2^8 growth), so O is rescaled in TMEM rarely;
+//   * the epilogue stages finished rows in the idle K/V rings and writes them out with coalesced
+//     16-byte stores.
 // Every mbarrier wait is bounded: on time-out the CTA records TSD_ERR_TIMEOUT, drains its own
 // TMA copies (again bounded) and frees its TMEM before returning.
 #include <cuda.h>
