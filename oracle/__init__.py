@@ -291,3 +291,4 @@ def verify_step(inp: dict, rows=None):
 
 
 from .draft_tree import DraftTree, draft_tree_build  # noqa: E402,F401
+from . import ssd_cache  # noqa: E402,F401
