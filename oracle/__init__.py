@@ -292,3 +292,4 @@ def verify_step(inp: dict, rows=None):
 
 from .draft_tree import DraftTree, draft_tree_build  # noqa: E402,F401
 from . import ssd_cache  # noqa: E402,F401
+from . import tree_sample  # noqa: E402,F401
