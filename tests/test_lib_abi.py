@@ -96,3 +96,15 @@ def test_host_checks_of_the_fused_and_draft_tree_entry_points():
     assert L.tsd_draft_tree_finalize(ctypes.byref(big), 0, 8, None, None, None, None, None) == 1      # > 4096 nodes
     # one record of (2 x 4 + 16) bytes rounded to 16, per (sequence, row, 16384-token chunk)
     assert tsd.lib().tsd_draft_tree_expand_workspace_size(2, 10, 10, 128256) == 2 * 10 * 8 * 96
+
+
+def test_split_planner_choices_for_the_bench_workloads():
+    """The planner's split counts (read back through the workspace size: splits * rows * (d + 2)
+    fp32 per KV head and sequence) for the four bench shapes on a 148-SM device; a split-count sweep
+    on B200 measured these as the fastest for tree26 (3..17) and eagle60 (1..4)."""
+    def splits(ws, B, Hkv, R, d=128):
+        return ws // (B * Hkv * R * (d + 2) * 4) if ws else 1
+    assert splits(tsd.tree_verify_attn_workspace_size(1, 26, 32, 8, 128, 2112, 1), 1, 8, 104) == 9
+    assert splits(tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1), 16, 8, 240) == 1
+    assert splits(tsd.tree_verify_attn_workspace_size(64, 6, 64, 8, 128, 8256, 1), 64, 8, 48) == 2
+    assert splits(tsd.tree_verify_attn_paged_workspace_size(8, 512, 32, 8, 128, 2080, 16, 1), 8, 8, 2048) == 2
