@@ -5,7 +5,12 @@ A step is the whole hot path over one batch: tree_prepare -> tree_verify_attn (+
 tokens per second (sum of tree nodes over the timed steps / device time), with the attention
 call's achieved HBM bandwidth against the measured copy bandwidth as the roofline figure.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload tree26] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+The headline line is the chain5 workload (the largest: 2.16 GB of attention K/V per step).  With
+no --workload at one GPU, the same measurement is also taken on the other four workloads and
+reported under "per_workload" (value, ms per step, roofline, e2e of each); --workload NAME
+measures that workload alone.
 
 Multi-GPU (torchrun): every rank verifies its own batch (its own seeded sequences), no
 collective on the data path; the timed region is bracketed by a barrier and a synchronize, the
@@ -33,7 +38,8 @@ import numpy as np  # noqa: E402
 import workloads as W  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
-DEFAULT_WORKLOAD = "tree26"
+DEFAULT_WORKLOAD = "chain5"
+ALL_WORKLOADS = ("tiny", "tree26", "eagle60", "chain5", "forest")
 DESCR = {
     "tiny": "B=1 Hq=8 Hkv=2 d=64 fp32, L=128, 8-node tree, V=256",
     "tree26": "Llama-3-8B-shaped verify: B=1 Hq=32 Hkv=8 d=128 bf16, L=2048, static EAGLE tree N=26 "
@@ -108,23 +114,34 @@ def aggregate_rate(tokens_per_rank_step: int, world: int, steps: int, max_ms: fl
     return world * tokens_per_rank_step * steps / (max_ms * 1e-3)
 
 
-def read_tensor_peak():
-    """Dense bf16 TFLOP/s: the measured burst cuBLAS figure (the attention graph times one kernel
-    back to back, and it does not reach the power cap), else the profiling recipe's fallback."""
+def _peaks_file():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
-            j = json.load(f)
-        if "bf16_tflops" in j:
-            return float(j["bf16_tflops"]), "measured bf16_tflops (cuBLAS, burst)"
+            return json.load(f)
+    return {}
+
+
+def read_tensor_peak():
+    """Dense bf16 TFLOP/s: the measured burst cuBLAS figure (the attention graph times one kernel
+    back to back for well under a second), else the profiling recipe's fallback."""
+    j = _peaks_file()
+    if "bf16_tflops" in j:
+        return float(j["bf16_tflops"]), "measured bf16_tflops (cuBLAS, burst)"
     return 1590.0, "fallback bf16 (burst)"
 
 
+def read_tensor_peak_sustained():
+    """Dense bf16 TFLOP/s sustained under the power cap (seconds-long cuBLAS loop)."""
+    j = _peaks_file()
+    if "bf16_tflops_sustained" in j:
+        return float(j["bf16_tflops_sustained"]), "measured bf16_tflops_sustained"
+    return 1400.0, "fallback bf16 (sustained)"
+
+
 def read_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            j = json.load(f)
+    j = _peaks_file()
+    if "hbm_gbs" in j:
         return float(j["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
 
@@ -207,16 +224,46 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
+def _roofline(inp, attn_ms, workload):
+    """Roofline of the attention call: its bound is whichever floor is higher, the algorithmic
+    bytes at the measured copy bandwidth or the algorithmic flops at the dense bf16 rate; both
+    fractions are reported, the tensor one against the burst and the sustained bf16 figures."""
+    peak, peak_kind = read_peaks()
+    tpeak, tpeak_kind = read_tensor_peak()
+    spk, spk_kind = read_tensor_peak_sustained()
+    alg = attn_algorithmic_bytes(inp)
+    flops = attn_algorithmic_flops(inp)
+    sec = attn_ms * 1e-3
+    tensor_bound = flops / (tpeak * 1e12) > alg / (peak * 1e9)
+    if tensor_bound:
+        roof = {"bound": "tensor", "achieved": round(flops / sec / 1e12, 1), "peak": tpeak, "unit": "TFLOP/s"}
+        roof["frac"] = round(roof["achieved"] / tpeak, 4)
+        roof["peak_kind"] = tpeak_kind + " (of measured)" if "measured" in tpeak_kind else tpeak_kind
+    else:
+        achieved = alg / sec / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"}
+    roof.update({"traffic": recorded_traffic(workload), "kernel": "tsd_tree_verify_attn",
+                 "algorithmic_bytes_per_launch": alg, "algorithmic_flops_per_launch": flops,
+                 "attn_us_per_launch": round(attn_ms * 1e3, 3),
+                 "hbm_frac": round(alg / sec / 1e9 / peak, 4),
+                 "tensor_frac": round(flops / sec / 1e12 / tpeak, 4),
+                 "tensor_frac_sustained": round(flops / sec / 1e12 / spk, 4),
+                 "tensor_peak_sustained": spk})
+    return roof
+
+
+def measure(name, args, rank, world, dev, gpu_id):
+    """One workload: K whole steps captured into one CUDA graph and timed with CUDA events (max over
+    ranks), the attention call alone the same way, and the e2e figure through the public API with
+    host buffers.  Returns (fields of the JSON line, the generated inputs)."""
     import torch
     import torch.distributed as dist
 
     import tree_speculative_decoding_06_b200 as tsd
     from tree_speculative_decoding_06_b200.step import VerifyStep, to_device
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w, seed = rank_workload(args.workload, rank, args.batch)
+    w, seed = rank_workload(name, rank, args.batch)
     inp = W.make_inputs(w, seed=seed, nan_guard=False)
     tok = tokens_per_step(inp)
     x0 = to_device(inp, dev)
@@ -237,6 +284,7 @@ def run_ours(args, rank, world, local_rank):
         for i in range(max(args.warmup, 3)):
             one_step(i)
     torch.cuda.synchronize(dev)
+
     # The timed K steps are captured into ONE CUDA graph (step i on input set i % nsets), so the
     # device runs them back to back with no per-step host launch cost; likewise K attention calls.
     def attn_call(s):
@@ -263,8 +311,6 @@ def run_ours(args, rank, world, local_rank):
         g_attn.replay()
     torch.cuda.synchronize(dev)
 
-    gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank] \
-        if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local_rank)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -289,9 +335,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     step_ms, attn_ms = reduce_over_ranks([step_ms, attn_ms], world, dev)
-
-    # status check: every sequence of every set must be clean
-    bad = sum(int((st.status != 0).sum()) for st in steps)
+    bad = sum(int((st.status != 0).sum()) for st in steps)   # every sequence of every set must be clean
 
     # end to end through the public API with host buffers: H2D of the step's inputs from pinned
     # memory, the step, D2H of the accepted lengths / tokens / path
@@ -303,88 +347,88 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(host[k].numel() * host[k].element_size() for k in keys_in)
     d2h = sum(host_out[k].numel() * host_out[k].element_size() for k in outs)
     e_steps = max(10, min(args.steps, 200))
+
+    def e2e_step():
+        for k in keys_in:
+            sets[0][k].copy_(host[k], non_blocking=True)
+        one_step(0)
+        for k in outs:
+            host_out[k].copy_(getattr(steps[0], k), non_blocking=True)
+
     with torch.cuda.stream(stream):
-        for i in range(3):
-            for k in keys_in:
-                sets[0][k].copy_(host[k], non_blocking=True)
-            one_step(0)
-            for k in outs:
-                host_out[k].copy_(getattr(steps[0], k), non_blocking=True)
+        for _ in range(3):
+            e2e_step()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for i in range(e_steps):
-            for k in keys_in:
-                sets[0][k].copy_(host[k], non_blocking=True)
-            one_step(0)
-            for k in outs:
-                host_out[k].copy_(getattr(steps[0], k), non_blocking=True)
+        for _ in range(e_steps):
+            e2e_step()
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e_ms = reduce_over_ranks([e0.elapsed_time(e1) / e_steps], world, dev)[0]
 
-    # launches of our kernels: per step (prepare, attention (+ merge), fused acceptance + commit,
-    # or the chain sampler and the commit), plus the attention-only graph
+    # launches of our kernels: per step (prepare, attention (+ merge), acceptance, commit), plus the
+    # attention-only graph
     per_step = steps[0].launches_per_step()
-    launches = per_step * args.steps + (1 + int(steps[0].splits_merge)) * n_attn
+    launches = per_step * args.steps + steps[0].attn_launches() * n_attn
+    fields = {
+        "value": round(aggregate_rate(tok, world, args.steps, step_ms), 1),
+        "ms_per_step": round(step_ms / args.steps, 6),
+        "dtype": "bf16" if inp["q"].dtype == np.uint16 else "f32",
+        "config": {"workload": f"{name}: {DESCR[name]}" +
+                               (f" [batch overridden to {args.batch}]" if args.batch else ""),
+                   "tokens_per_step_per_gpu": tok,
+                   "l2": (f"rotating {nsets} input sets ({nsets * per_set / 2**20:.0f} MiB > 2x L2)"
+                          if nsets > 1 else f"inputs {per_set / 2**20:.0f} MiB > L2"),
+                   "graphs": "the K timed steps replayed as one CUDA graph",
+                   "parallelism": f"replicas over sequences x{world}"},
+        "roofline": _roofline(inp, attn_ms, name) if rank == 0 else None,
+        "e2e": {"value": round(aggregate_rate(tok, world, 1, e_ms), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+        "status_errors": bad,
+        "wall_s_timed": round(wall, 3),
+    }
+    del g_steps, g_attn, sets, steps, x0, host, host_out
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return fields, inp
 
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank] \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local_rank)
+    head = args.workload or DEFAULT_WORKLOAD
+    fields, inp = measure(head, args, rank, world, dev, gpu_id)
     res = None
     if rank == 0:
-        peak, peak_kind = read_peaks()
-        tpeak, tpeak_kind = read_tensor_peak()
-        alg = attn_algorithmic_bytes(inp)
-        flops = attn_algorithmic_flops(inp)
-        traffic = recorded_traffic(args.workload)
-        # the bound is whichever floor is higher: the bytes at the copy bandwidth or the flops at
-        # the dense bf16 rate
-        tensor_bound = flops / (tpeak * 1e12) > alg / (peak * 1e9)
-        if tensor_bound:
-            roof = {"bound": "tensor", "achieved": round(flops / (attn_ms * 1e-3) / 1e12, 1), "peak": tpeak,
-                    "unit": "TFLOP/s"}
-            roof["frac"] = round(roof["achieved"] / tpeak, 4)
-            roof["peak_kind"] = tpeak_kind
-        else:
-            achieved = alg / (attn_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"}
-        roof.update({"traffic": traffic, "kernel": "tsd_tree_verify_attn (split kernel + merge)",
-                     "algorithmic_bytes_per_launch": alg, "algorithmic_flops_per_launch": flops,
-                     "attn_us_per_launch": round(attn_ms * 1e3, 3),
-                     "hbm_frac": round(alg / (attn_ms * 1e-3) / 1e9 / peak, 4),
-                     "tensor_frac": round(flops / (attn_ms * 1e-3) / 1e12 / tpeak, 4)})
-        value = aggregate_rate(tok, world, args.steps, step_ms)
-        res = {
-            "metric": METRIC,
-            "value": round(value, 1),
-            "unit": "tokens/s",
-            "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup,
-            "ms_per_step": round(step_ms / args.steps, 6),
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "bf16" if inp["q"].dtype == np.uint16 else "f32",
-            "data": "synthetic (seeded; workloads module)",
-            "config": {"workload": f"{args.workload}: {DESCR[args.workload]}" +
-                                   (f" [batch overridden to {args.batch}]" if args.batch else ""),
-                       "tokens_per_step_per_gpu": tok,
-                       "l2": (f"rotating {nsets} input sets ({nsets * per_set / 2**20:.0f} MiB > 2x L2)"
-                              if nsets > 1 else f"inputs {per_set / 2**20:.0f} MiB > L2"),
-                       "graphs": "the K timed steps replayed as one CUDA graph",
-                       "parallelism": f"replicas over sequences x{world}"},
-            "roofline": roof,
-            "e2e": {"value": round(aggregate_rate(tok, world, 1, e_ms), 1), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": round(e_ms, 4)},
-            "gpu_launches": launches,
-            "clocks": clocks.summary(),
-            "status_errors": bad,
-            "wall_s_timed": round(wall, 3),
-        }
+        res = {"metric": METRIC, "value": fields["value"], "unit": "tokens/s", "n_gpus": world,
+               "steps": args.steps, "warmup": args.warmup, "ms_per_step": fields["ms_per_step"],
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": fields["dtype"],
+               "data": "synthetic (seeded; workloads module)"}
+        res.update({k: fields[k] for k in ("config", "roofline", "e2e", "gpu_launches", "clocks", "status_errors",
+                                           "wall_s_timed")})
+    # every other workload at one GPU when none was named: same measurement, reported per workload
+    if args.workload is None and world == 1:
+        per = {}
+        for name in ALL_WORKLOADS:
+            if name == head:
+                continue
+            f, _ = measure(name, args, rank, world, dev, gpu_id)
+            per[name] = {k: f[k] for k in ("value", "ms_per_step", "dtype", "roofline", "e2e", "gpu_launches",
+                                           "clocks", "status_errors")}
+            per[name]["unit"] = "tokens/s"
+            per[name]["workload"] = f["config"]["workload"]
+            res["gpu_launches"] += f["gpu_launches"]
+        res["per_workload"] = per
     return res, inp
 
 
@@ -438,7 +482,8 @@ def run_reference(args, rank):
         return None
     import oracle
     oracle.build()
-    w = W.WORKLOADS[args.workload]
+    name = args.workload or DEFAULT_WORKLOAD
+    w = W.WORKLOADS[name]
     inp = W.make_inputs(w, nan_guard=False)
     for _ in range(max(args.warmup, 0)):
         oracle_sample(inp, 0.0)
@@ -449,14 +494,14 @@ def run_reference(args, rank):
         secs += dt
     value = float(np.mean(rates))
     step_tokens = tokens_per_step(inp)
-    cb = {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+    cb = {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle", "host_cores": os.cpu_count(),
           "sample": f"per step: {desc}; {args.steps} steps, {secs:.1f} s"}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 2),
             "unit": "tokens/s", "n_gpus": args.gpus, "ran_on": "one host core of rank 0 (the fp64 oracle)",
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(step_tokens / value * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; workloads module)",
-            "config": {"workload": f"{args.workload}: {DESCR[args.workload]}", "tokens_per_step_per_gpu": step_tokens},
+            "config": {"workload": f"{name}: {DESCR[name]}", "tokens_per_step_per_gpu": step_tokens},
             "cpu_baseline": cb,
             "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -467,7 +512,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(W.WORKLOADS),
+                    help="measure this workload alone (default: the chain5 headline plus, at one GPU, every "
+                         "other workload under per_workload)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--batch", type=int, default=0,
@@ -497,6 +544,7 @@ def main():
             if world == 1:   # the oracle baseline is timed at one GPU only
                 v, desc, dt = oracle_sample(inp, args.cpu_budget)
                 res["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                       "host_cores": os.cpu_count(),
                                        "sample": f"{desc}; {dt:.1f} s, single-threaded C fp64"}
                 res["speedup_vs_cpu_baseline"] = round(res["value"] / v, 1)
             print(json.dumps(res))

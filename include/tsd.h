@@ -39,6 +39,12 @@
  *       k/v_pages     [num_blocks, Hkv, block_size, d] + block_table [B, max_blocks] (int32)
  *       logits        [B, Nmax, V]             (dtype)
  *     Q and K are taken after the positional encoding (RoPE) has been applied by the caller.
+ *   - Alignment: every tensor pointer an entry point moves in 16-byte pieces (Q, K, V, O and
+ *     the caches of the attention, the caches and tree K/V of the commit, every workspace) must
+ *     be 16-byte aligned, else the call returns TSD_ERR_INVALID_ARG (TSD_ERR_WORKSPACE for a
+ *     workspace) before any launch.  Logits may start anywhere: the vocabulary scans take their
+ *     16-byte path only when the base pointer is 16-byte aligned and V % 8 == 0, and read one
+ *     element at a time otherwise.
  *   - Return value: host-detected problems (null pointers, bad sizes, unsupported dtypes, a
  *     too small workspace, launch failures).  Problems that only the device can see
  *     (a malformed tree, a prefix past the cache capacity, a bad block-table entry, a bad
@@ -68,7 +74,7 @@ typedef enum tsd_status {
     TSD_ERR_TREE_DEPTH = 4,        /* depth(i) > Dmax: depth consistency ([EP] sec. 2) */
     TSD_ERR_TREE_ROOTS = 5,        /* a second root outside forest mode */
     TSD_ERR_CAPACITY = 6,          /* prefix + rows beyond the cache (or block table) capacity */
-    TSD_ERR_TIMEOUT = 7,           /* reserved for bounded device waits (none in this version) */
+    TSD_ERR_TIMEOUT = 7,           /* a bounded device wait gave up (tcgen05 attention pipeline) */
     TSD_ERR_CUDA = 8,              /* a kernel launch failed (cudaGetLastError) */
     TSD_ERR_WORKSPACE = 9          /* workspace pointer null or smaller than the query said */
 } tsd_status;
@@ -213,11 +219,17 @@ tsd_status tsd_tree_accept_greedy(const void *logits, tsd_dtype dtype, int V, co
  *     TSD_ACCEPT_NOALLOC_SCRATCH_BYTES is refused with TSD_ERR_WORKSPACE before any launch
  *     (1 MiB holds e.g. B*Nmax = 8192 rows of a 128256-token vocabulary).
  *   - The first call on a device looks up the array's device address (with that device
- *     current) and caches it; make that first call before any stream capture.
+ *     current) and caches it; make that first call before any stream capture.  The cached
+ *     address belongs to the device's primary context: after cudaDeviceReset on that device
+ *     the library must be reloaded before this call is used again.
  *   - Every call shares the one array: calls that overlap on the GPU (other streams, other
  *     host threads) race and must be serialised by the caller.
  * --------------------------------------------------------------------------------------- */
 #define TSD_ACCEPT_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* Size of that fixed array as compiled into the loaded library (equals
+ * TSD_ACCEPT_NOALLOC_SCRATCH_BYTES of the header it was built with). */
+size_t tsd_tree_accept_greedy_noalloc_scratch_bytes(void);
 
 tsd_status tsd_tree_accept_greedy_noalloc(const void *logits, tsd_dtype dtype, int V, const int32_t *tokens,
                                           const int32_t *parent_s, const int32_t *num_nodes,

@@ -44,7 +44,7 @@ def test_accept_greedy_full(name):
     ref = oracle.accept_greedy(inp)
     assert_accept_equal(got, ref)
     if name == "forest":   # the fixture hits some roots and misses others
-        assert (ref["accept_len"] == -1).any() or True
+        assert (ref["accept_len"] == -1).any() and (ref["accept_len"] >= 0).any()
 
 
 def test_accept_greedy_edge_cases():
@@ -116,11 +116,34 @@ def final_interval_distance(zp, zq, u, T, b, j, tok):
     return 0.0 if lo <= thr < hi else min(abs(thr - lo), abs(thr - hi)) / R
 
 
-def compare_sampling(got, ref, K, zp=None, zq=None, u=None, T=None):
-    """Bit-exact on every sequence whose decisions all clear their margins; a sequence whose
-    final draw is near a boundary must still agree on every accept decision and draw a token
-    whose cumulative interval lies within CDF_MARGIN of the threshold.  Returns the number of
-    near-boundary sequences."""
+def final_distribution_mass(zp, zq, T, b, j, tok):
+    """fp64 mass of `tok` under the distribution the final draw at position j samples from: the
+    residual max(p_j - q_j, 0) after a rejection at j < K (p_j if that residual is empty), p_K
+    when every draft was accepted.  A drawn token must have positive mass there."""
+    dt = "bf16" if zp.dtype == np.uint16 else "f32"
+    K = zq.shape[1]
+    zpj = W.as_f32(zp[b, j], dt).astype(np.float64) / T
+    p = np.exp(zpj - zpj.max())
+    p /= p.sum()
+    if j == K:
+        return float(p[tok])
+    zqj = W.as_f32(zq[b, j], dt).astype(np.float64) / T
+    q = np.exp(zqj - zqj.max())
+    q /= q.sum()
+    r = np.maximum(p - q, 0.0)
+    return float(r[tok] if r.sum() > 0 else p[tok])
+
+
+def compare_sampling(got, ref, K, zp=None, zq=None, u=None, T=None, x=None):
+    """Bit-exact on every sequence whose decisions all clear their margins.  A sequence with a
+    decision near its margin is checked for validity instead:
+      * accept tests: every test before the first near one clears its margin, so the kernel must
+        accept exactly as the oracle did up to there (A >= that index); the A emitted tokens
+        before the draw are the drafts x[:A]; the drawn token has positive fp64 mass under the
+        distribution the draw at A samples from; every entry past A is -1;
+      * a near final draw with clear tests: the same accept decisions, and a token whose
+        cumulative interval lies within CDF_MARGIN of the threshold.
+    Returns the number of near-margin sequences."""
     m = ref["margin"]
     acc_near = (m[:, :K] < ACC_MARGIN).any(1)
     cdf_near = m[:, K] < CDF_MARGIN
@@ -129,6 +152,20 @@ def compare_sampling(got, ref, K, zp=None, zq=None, u=None, T=None):
     assert np.array_equal(got["out_tokens"][far], ref["out_tokens"][far])
     A = got["accept_len"]
     assert ((A >= 0) & (A <= K)).all()
+    for b in np.nonzero(acc_near)[0]:
+        j0 = int(np.nonzero(m[b, :K] < ACC_MARGIN)[0][0])
+        a = int(A[b])
+        assert a >= j0, (b, a, j0)
+        if x is not None:
+            assert np.array_equal(got["out_tokens"][b, :a], x[b, :a])
+        else:
+            n = min(a, int(ref["accept_len"][b]))
+            assert np.array_equal(got["out_tokens"][b, :n], ref["out_tokens"][b, :n])
+        assert (got["out_tokens"][b, a + 1:] == -1).all()
+        tok = int(got["out_tokens"][b, a])
+        assert 0 <= tok < (zp.shape[2] if zp is not None else np.iinfo(np.int32).max)
+        if zp is not None:
+            assert final_distribution_mass(zp, zq, T, b, a, tok) > 0.0, (b, a, tok)
     for b in np.nonzero(cdf_near & ~acc_near)[0]:
         j = int(ref["accept_len"][b])
         assert got["accept_len"][b] == j
@@ -142,7 +179,7 @@ def test_chain_sample_full_size():
     inp = W.make_inputs(W.WORKLOADS["chain5"])
     got = gpu_sample(inp["z_p"], inp["z_q"], inp["x"], inp["u"], 1.0)
     ref = oracle.chain_sample(inp["z_p"], inp["z_q"], inp["x"], inp["u"], 1.0)
-    n_near = compare_sampling(got, ref, 5, inp["z_p"], inp["z_q"], inp["u"], 1.0)
+    n_near = compare_sampling(got, ref, 5, inp["z_p"], inp["z_q"], inp["u"], 1.0, inp["x"])
     assert n_near <= 2
     assert len(set(ref["accept_len"].tolist())) > 1   # the fixture exercises several accepted lengths
 
@@ -162,7 +199,7 @@ def test_chain_sample_small(V, dt):
     for T in (1.0, 0.7):
         got = gpu_sample(zp, zq, x, u, T)
         ref = oracle.chain_sample(zp, zq, x, u, T)
-        assert compare_sampling(got, ref, K, zp, zq, u, T) <= 3
+        assert compare_sampling(got, ref, K, zp, zq, u, T, x) <= 3
     got = gpu_sample(zp, zq, x, u, 0.0)
     ref = oracle.chain_sample(zp, zq, x, u, 0.0)
     assert np.array_equal(got["accept_len"], ref["accept_len"])
@@ -288,30 +325,92 @@ def test_commit_errors_leave_cache_untouched():
 
 
 # ----------------------------------------------------------------------------- whole step
+_STEP_CASES = {}
+
+
+def _step_case(name):
+    """Inputs of the whole-step test and the oracle's outputs on them (attention of every row,
+    acceptance, commit), computed once per workload and shared by the three schedules."""
+    if name not in _STEP_CASES:
+        w = W.WORKLOADS[name]
+        if name == "forest":       # 2 x 512 nodes x 32 heads: every row is checked
+            w = w.scaled(B=2, L=700)
+        elif name in ("chain5", "eagle60"):
+            w = w.scaled(B=min(w.B, 4), L=min(w.L, 3000), L_lo=None if w.L_lo is None else 500)
+        inp = W.make_inputs(w, nan_guard=False)
+        att = oracle.attention_rows(inp)
+        if w.accept == "greedy":
+            acc = oracle.accept_greedy(inp)
+            com = oracle.kv_commit(inp, acc["accept_len"], acc["path"], "path")
+        else:
+            acc = oracle.chain_sample(inp["z_p"], inp["z_q"], inp["x"], inp["u"], inp["T"])
+            com = oracle.kv_commit(inp, acc["accept_len"], None, "length")
+        _STEP_CASES[name] = (w, inp, att, acc, com)
+    return _STEP_CASES[name]
+
+
+def _bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.cpu().numpy()
+
+
 @pytest.mark.parametrize("name,schedule", [(n, s) for n in ("tiny", "tree26", "eagle60", "forest")
                                             for s in ("overlap", "fused", "serial")] + [("chain5", None)])
 def test_verify_step_matches_oracle(name, schedule):
-    w = W.WORKLOADS[name]
-    if name in ("chain5", "forest", "eagle60"):
-        w = w.scaled(B=min(w.B, 4), L=min(w.L, 3000), L_lo=None if w.L_lo is None else 500)
-    inp = W.make_inputs(w, nan_guard=False)
+    """The whole step under each schedule: the attention output of every row within tolerance,
+    acceptance bit-exact (margin protocol for sampling), and the K and V caches byte-exact after
+    the commit (guard rows included), with prefix_len advanced as the oracle's commit does."""
+    from gpu_helpers import TOL
+    w, inp, (ref_o, _, rows), ref, (rk, rv, rpl, _) = _step_case(name)
     x = to_device(inp)
     step = VerifyStep.for_inputs(x, schedule=schedule)
     res = step.run(x)
     torch.cuda.synchronize()
     assert (res["status"].cpu().numpy() == 0).all()
+    out = res["out"].float().cpu().numpy().astype(np.float64)
+    got_o = np.stack([out[b, i, h] for (b, i, h) in rows])
+    atol, rtol = TOL["bf16" if w.dtype == "bf16" else "f32"]
+    assert not np.isnan(got_o).any()
+    assert (np.abs(got_o - ref_o) <= atol + rtol * np.abs(ref_o)).all(), np.abs(got_o - ref_o).max()
     if w.accept == "greedy":
-        ref = oracle.accept_greedy(inp)
         assert np.array_equal(res["accept_len"].cpu().numpy(), ref["accept_len"])
+        assert np.array_equal(res["path"].cpu().numpy(), ref["path"])
         assert np.array_equal(res["out_tokens"].cpu().numpy(), ref["out_tokens"])
-        rk, rv, rpl, _ = oracle.kv_commit(inp, ref["accept_len"], ref["path"], "path")
     else:
-        ref = oracle.chain_sample(inp["z_p"], inp["z_q"], inp["x"], inp["u"], inp["T"])
         got = {"accept_len": res["accept_len"].cpu().numpy(), "out_tokens": res["out_tokens"].cpu().numpy()}
-        assert compare_sampling(got, ref, w.K, inp["z_p"], inp["z_q"], inp["u"], inp["T"]) <= 1
-        rk, rv, rpl, _ = oracle.kv_commit(inp, ref["accept_len"], None, "length")
+        assert compare_sampling(got, ref, w.K, inp["z_p"], inp["z_q"], inp["u"], inp["T"], inp["x"]) <= 1
+        if not np.array_equal(got["accept_len"], ref["accept_len"]):
+            pytest.skip("a near-margin sampling decision differs from the oracle's: caches not comparable")
     assert np.array_equal(x["prefix_len"].cpu().numpy(), rpl)
-    key = "k_pages" if w.paged else "k_cache"
-    got_k = x[key].view(torch.int16).cpu().numpy().view(np.uint16) if x[key].dtype == torch.bfloat16 else \
-        x[key].cpu().numpy()
-    assert np.array_equal(got_k, rk)
+    kkey, vkey = ("k_pages", "v_pages") if w.paged else ("k_cache", "v_cache")
+    assert np.array_equal(_bits(x[kkey]), rk)
+    assert np.array_equal(_bits(x[vkey]), rv)
+
+
+def test_schedules_agree_on_a_sequence_the_attention_flags():
+    """A bad block id inside one sequence's prefix makes the attention flag that sequence
+    (TSD_ERR_CAPACITY) while the acceptance may already be running on the side stream.  Every
+    schedule must leave the same status, caches and prefix lengths, the flagged sequence's cache
+    untouched and its attention rows zero, and agree with the oracle on the other sequences."""
+    w = W.WORKLOADS["eagle60"].scaled(B=3, L=600, L_lo=300)
+    inp = W.make_inputs(w, nan_guard=False)
+    bad_b = 1
+    inp["block_table"] = inp["block_table"].copy()
+    inp["block_table"][bad_b, 2] = 1 << 30              # inside its prefix: prefix_len >= 300 > 2 * 16
+    ref = oracle.accept_greedy(inp)
+    outcomes = []
+    for schedule in ("overlap", "fused", "serial"):
+        x = to_device(inp)
+        step = VerifyStep.for_inputs(x, schedule=schedule)
+        res = step.run(x)
+        torch.cuda.synchronize()
+        st = res["status"].cpu().numpy()
+        assert (st & 0xFF).tolist() == [0 if b != bad_b else 6 for b in range(w.B)], st
+        good = st == 0
+        assert np.array_equal(res["accept_len"].cpu().numpy()[good], ref["accept_len"][good])
+        assert np.array_equal(res["out_tokens"].cpu().numpy()[good], ref["out_tokens"][good])
+        assert (res["out"][bad_b].float() == 0).all()
+        outcomes.append((st, x["prefix_len"].cpu().numpy(), _bits(x["k_pages"]), _bits(x["v_pages"])))
+    for o in outcomes[1:]:
+        for a, b in zip(outcomes[0], o):
+            assert np.array_equal(a, b)
+    assert outcomes[0][1][bad_b] == inp["prefix_len"][bad_b]

@@ -108,3 +108,29 @@ def test_split_planner_choices_for_the_bench_workloads():
     assert splits(tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1), 16, 8, 240) == 1
     assert splits(tsd.tree_verify_attn_workspace_size(64, 6, 64, 8, 128, 8256, 1), 64, 8, 48) == 2
     assert splits(tsd.tree_verify_attn_paged_workspace_size(8, 512, 32, 8, 128, 2080, 16, 1), 8, 8, 2048) == 2
+
+
+def test_misaligned_tensor_pointers_are_refused_before_any_launch():
+    """Every pointer the kernels move in 16-byte pieces must be 16-byte aligned; a view at an odd
+    storage offset is refused with a status code on the host instead of reaching a kernel."""
+    L = tsd.lib()
+    buf = ctypes.create_string_buffer(1 << 16)
+    base = (ctypes.addressof(buf) + 255) & ~255
+    p, odd = ctypes.c_void_p(base), ctypes.c_void_p(base + 4)
+    ws = tsd.tree_verify_attn_workspace_size(1, 26, 32, 8, 128, 2112, 1)
+    # attention: Q, a cache or the output off a 16-byte boundary -> INVALID_ARG; workspace -> WORKSPACE
+    for i in (0, 1, 2, 5, 6, 17):
+        a = [p] * 23
+        a[i] = odd
+        rc = L.tsd_tree_verify_attn(a[0], a[1], a[2], 2112, p, a[5], a[6], p, None, 1, 26, 32, 8, 128, 6, 1, 0.1,
+                                    a[17], None, p, ws, p, None)
+        assert rc == 1, i
+    assert L.tsd_tree_verify_attn(p, p, p, 2112, p, p, p, p, None, 1, 26, 32, 8, 128, 6, 1, 0.1, p, None, odd, ws,
+                                  p, None) == 9
+    # commit: cache or tree rows off a 16-byte boundary
+    assert L.tsd_kv_commit(odd, p, 16, p, p, p, p, p, None, 1, 4, 2, 64, 3, 1, 0, p, None) == 1
+    assert L.tsd_kv_commit(p, p, 16, p, odd, p, p, p, None, 1, 4, 2, 64, 3, 1, 0, p, None) == 1
+    # acceptance workspace
+    need = tsd.tree_accept_greedy_workspace_size(1, 4, 64)
+    assert L.tsd_tree_accept_greedy(p, 1, 64, p, p, None, None, 1, 4, 3, p, p, p, odd, need, p, None) == 9
+    assert tsd.accept_noalloc_scratch_bytes() == 1 << 20

@@ -41,7 +41,7 @@ def test_noalloc_equals_workspace_call_on_consecutive_calls():
 
 def test_noalloc_refuses_batches_beyond_its_scratch():
     B, Nmax, V = 16, 600, 128256           # 16*600 rows x 16 chunks x 8 B > 1 MiB
-    assert tsd.tree_accept_greedy_workspace_size(B, Nmax, V) > tsd.ACCEPT_NOALLOC_SCRATCH_BYTES
+    assert tsd.tree_accept_greedy_workspace_size(B, Nmax, V) > tsd.accept_noalloc_scratch_bytes()
     logits = torch.zeros(1, dtype=torch.bfloat16, device="cuda")
     i32 = torch.zeros(1, dtype=torch.int32, device="cuda")
     p = ctypes.c_void_p(i32.data_ptr())

@@ -44,6 +44,7 @@ _SIGS = {
     "tsd_tree_accept_greedy_workspace_size": (_SZ, [_I, _I, _I]),
     "tsd_tree_accept_greedy": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_accept_greedy_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "tsd_tree_accept_greedy_noalloc_scratch_bytes": (_SZ, []),
     "tsd_chain_accept_sample_workspace_size": (_SZ, [_I, _I, _I]),
     "tsd_chain_accept_sample": (_I, [_P, _P, _I, _I, _P, _P, _F, _I, _I, _P, _P, _P, _SZ, _P]),
     "tsd_kv_commit": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -241,13 +242,15 @@ def tree_accept_greedy(logits, tokens, parent_s, num_nodes=None, root_key=None, 
     return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
 
 
-ACCEPT_NOALLOC_SCRATCH_BYTES = 1 << 20
+def accept_noalloc_scratch_bytes() -> int:
+    """Size of the fixed scratch array tree_accept_greedy_noalloc uses, read from the library."""
+    return int(lib().tsd_tree_accept_greedy_noalloc_scratch_bytes())
 
 
 def tree_accept_greedy_noalloc(logits, tokens, parent_s, num_nodes=None, root_key=None, Dmax: int = 8,
                                accept_len=None, path=None, out_tokens=None, status=None, stream=None):
     """tree_accept_greedy for callers that may not allocate device scratch: the library's own
-    fixed scratch array (ACCEPT_NOALLOC_SCRATCH_BYTES per device) is used instead of a
+    fixed scratch array (accept_noalloc_scratch_bytes() per device) is used instead of a
     workspace.  Calls that overlap on the GPU share that array and race; the first call on a
     device should come before any stream capture."""
     B, Nmax, V = logits.shape

@@ -59,7 +59,7 @@ __device__ __forceinline__ void block_argmax(float& bv, int& bi) {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) row_argmax_chunks(const T* __restrict__ logits, int V, int rows_per_seq,
                                                               const int32_t* __restrict__ num_rows, int chunks,
-                                                              float2* __restrict__ part) {
+                                                              float2* __restrict__ part, int vec) {
   pdl_trigger();
   const int c = blockIdx.x, i = blockIdx.y, b = blockIdx.z;
   const int n = num_rows ? num_rows[b] : rows_per_seq;
@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kThreads) row_argmax_chunks(const T* __restric
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
   float bv = -INFINITY;
   int bi = INT_MAX;
-  if ((V & 7) == 0) {
+  if (vec) {
     for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
       float x[8];
       load8<T>(row, v, x);
@@ -145,12 +145,13 @@ tsd_status launch_row_argmax(const void* logits, tsd_dtype dtype, int V, int row
   const int chunks = num_chunks(V);
   float2* part = reinterpret_cast<float2*>(ws);
   dim3 grid(chunks, rows_per_seq, B);
+  const int vec = vec16_rows(logits, V) ? 1 : 0;
   if (dtype == TSD_BF16)
     launch_pdl(row_argmax_chunks<__nv_bfloat16>, grid, dim3(kThreads), 0, stream,
-               reinterpret_cast<const __nv_bfloat16*>(logits), V, rows_per_seq, num_rows, chunks, part);
+               reinterpret_cast<const __nv_bfloat16*>(logits), V, rows_per_seq, num_rows, chunks, part, vec);
   else
     launch_pdl(row_argmax_chunks<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(logits), V,
-               rows_per_seq, num_rows, chunks, part);
+               rows_per_seq, num_rows, chunks, part, vec);
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }
 
@@ -185,12 +186,13 @@ tsd_status launch_chain_sample(const void* zp, const void* zq, tsd_dtype dtype, 
   const int chunks = num_chunks(V);
   float2* part = reinterpret_cast<float2*>(ws);
   dim3 grid(chunks, K + 1, B);
+  const int vec = vec16_rows(zp, V) ? 1 : 0;
   if (dtype == TSD_BF16)
     launch_pdl(row_argmax_chunks<__nv_bfloat16>, grid, dim3(kThreads), 0, stream,
-               reinterpret_cast<const __nv_bfloat16*>(zp), V, K + 1, (const int32_t*)nullptr, chunks, part);
+               reinterpret_cast<const __nv_bfloat16*>(zp), V, K + 1, (const int32_t*)nullptr, chunks, part, vec);
   else
     launch_pdl(row_argmax_chunks<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(zp), V, K + 1,
-               (const int32_t*)nullptr, chunks, part);
+               (const int32_t*)nullptr, chunks, part, vec);
   launch_pdl(chain_greedy_decide, dim3((B + 127) / 128), dim3(128), 0, stream, (const float2*)part, chunks, x, B, K,
              accept_len, out_tokens);
   return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;

@@ -31,6 +31,8 @@ tsd_status check_attn_common(const void* q, const int32_t* prefix_len, const voi
   if (Dmax < 0 || Dmax > 255) return TSD_ERR_INVALID_ARG;
   if ((k_tree == nullptr) != (v_tree == nullptr)) return TSD_ERR_INVALID_ARG;
   if (B > 0 && Nmax > 0 && (!q || !prefix_len || !parent_s || !out || !status)) return TSD_ERR_INVALID_ARG;
+  // the kernels move Q, K, V and O rows in 16-byte pieces
+  if (!aligned16(q) || !aligned16(k_tree) || !aligned16(v_tree) || !aligned16(out)) return TSD_ERR_INVALID_ARG;
   return TSD_OK;
 }
 
@@ -88,8 +90,9 @@ tsd_status tsd_tree_verify_attn(const void* q, const void* k_cache, const void* 
   if (Lmax < 0) return TSD_ERR_INVALID_ARG;
   if (B == 0 || Nmax == 0) return TSD_OK;
   if (Lmax > 0 && (!k_cache || !v_cache)) return TSD_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return TSD_ERR_INVALID_ARG;
   const size_t need = tsd_tree_verify_attn_workspace_size(B, Nmax, Hq, Hkv, d, Lmax, dtype);
-  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return TSD_ERR_WORKSPACE;
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace))) return TSD_ERR_WORKSPACE;
   AttnArgs a{};
   a.q = q, a.k_cache = k_cache, a.v_cache = v_cache, a.block_table = nullptr;
   a.max_blocks = 0, a.block_shift = 0, a.num_blocks = 0, a.Lcap = Lmax, a.prefix_len = prefix_len;
@@ -113,9 +116,10 @@ tsd_status tsd_tree_verify_attn_paged(const void* q, const void* k_pages, const 
   if ((long long)max_blocks * block_size > 0x7fffffffLL) return TSD_ERR_INVALID_ARG;
   if (B == 0 || Nmax == 0) return TSD_OK;
   if (max_blocks > 0 && (!k_pages || !v_pages || !block_table)) return TSD_ERR_INVALID_ARG;
+  if (!aligned16(k_pages) || !aligned16(v_pages)) return TSD_ERR_INVALID_ARG;
   const size_t need =
       tsd_tree_verify_attn_paged_workspace_size(B, Nmax, Hq, Hkv, d, max_blocks, block_size, dtype);
-  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return TSD_ERR_WORKSPACE;
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace))) return TSD_ERR_WORKSPACE;
   AttnArgs a{};
   a.q = q, a.k_cache = k_pages, a.v_cache = v_pages, a.block_table = block_table;
   a.max_blocks = max_blocks, a.block_shift = log2i(block_size), a.num_blocks = num_blocks;
@@ -142,7 +146,7 @@ tsd_status tsd_tree_accept_greedy(const void* logits, tsd_dtype dtype, int V, co
   if (!accept_len || !path || !out_tokens || !status || !parent_s || (Nmax > 0 && (!logits || !tokens)))
     return TSD_ERR_INVALID_ARG;
   const size_t need = tsd_tree_accept_greedy_workspace_size(B, Nmax, V);
-  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return TSD_ERR_WORKSPACE;
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace))) return TSD_ERR_WORKSPACE;
   return launch_accept_greedy(logits, dtype, V, tokens, parent_s, num_nodes, root_key, B, Nmax, Dmax, accept_len,
                               path, out_tokens, workspace, status, S(stream));
 }
@@ -167,6 +171,8 @@ tsd_status tsd_tree_accept_greedy_noalloc(const void* logits, tsd_dtype dtype, i
                               path, out_tokens, scratch, status, S(stream));
 }
 
+size_t tsd_tree_accept_greedy_noalloc_scratch_bytes(void) { return (size_t)TSD_ACCEPT_NOALLOC_SCRATCH_BYTES; }
+
 size_t tsd_chain_accept_sample_workspace_size(int B, int K, int V) {
   if (B <= 0 || K < 0 || V <= 0) return 0;
   return chain_sample_ws(B, K, V);
@@ -182,7 +188,7 @@ tsd_status tsd_chain_accept_sample(const void* target_logits, const void* draft_
   if (!target_logits || !uniforms || !accept_len || !out_tokens || (K > 0 && (!draft_logits || !draft_tokens)))
     return TSD_ERR_INVALID_ARG;
   const size_t need = tsd_chain_accept_sample_workspace_size(B, K, V);
-  if (workspace == nullptr || ws_bytes < need) return TSD_ERR_WORKSPACE;
+  if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return TSD_ERR_WORKSPACE;
   return launch_chain_sample(target_logits, draft_logits, dtype, V, draft_tokens, uniforms, temperature, B, K,
                              accept_len, out_tokens, workspace, S(stream));
 }
@@ -198,6 +204,9 @@ static tsd_status commit_common(CommitArgs& a, const void* k_tree, const void* v
   if (!a.k_cache || !a.v_cache || !a.prefix_len || !accept_len || !a.status) return TSD_ERR_INVALID_ARG;
   if (mode != TSD_COMMIT_LENGTH && !path) return TSD_ERR_INVALID_ARG;
   if (mode != TSD_COMMIT_INPLACE && (!k_tree || !v_tree)) return TSD_ERR_INVALID_ARG;
+  // rows are copied in 16-byte pieces
+  if (!aligned16(a.k_cache) || !aligned16(a.v_cache) || !aligned16(k_tree) || !aligned16(v_tree))
+    return TSD_ERR_INVALID_ARG;
   a.k_tree = k_tree, a.v_tree = v_tree, a.path = path, a.accept_len = accept_len;
   a.esize = dtype == TSD_BF16 ? 2 : 4;
   a.mode = (int)mode;
@@ -270,7 +279,7 @@ tsd_status tsd_tree_accept_commit(const void* logits, tsd_dtype logits_dtype, in
     return TSD_ERR_INVALID_ARG;
   if (history && (history_cap < 0 || !history_len)) return TSD_ERR_INVALID_ARG;
   const size_t need = tsd_tree_accept_greedy_workspace_size(B, Nmax, V);
-  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return TSD_ERR_WORKSPACE;
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace))) return TSD_ERR_WORKSPACE;
   SpliceArgs sp{history, history_cap, history_len};
   return launch_accept_commit(logits, logits_dtype, V, tokens, parent_s, root_key, accept_len, path, out_tokens, a, sp,
                               workspace, S(stream));
@@ -310,7 +319,7 @@ tsd_status tsd_draft_tree_expand(const tsd_draft_tree* tree, const void* draft_l
   if (B == 0) return TSD_OK;
   if (!draft_logits || !status) return TSD_ERR_INVALID_ARG;
   const size_t need = draft_expand_ws(B, t.F, K, V);
-  if (workspace == nullptr || ws_bytes < need) return TSD_ERR_WORKSPACE;
+  if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return TSD_ERR_WORKSPACE;
   return launch_draft_expand(t, draft_logits, dtype, V, K, workspace, status, S(stream));
 }
 

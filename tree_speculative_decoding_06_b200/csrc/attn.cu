@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(256, 1)
   cp_async_wait<0>();
   __syncthreads();
   const bool err = s_err != 0;
-  if (err && split == 0 && mt == 0 && g == 0 && tid == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
+  if (err && tid == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
   if (!warp_on) return;
   lA += __shfl_xor_sync(0xffffffffu, lA, 1);
   lA += __shfl_xor_sync(0xffffffffu, lA, 2);
@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a, int BM,
   }
   __syncthreads();
   const bool err = s_err != 0;
-  if (err && split == 0 && mt == 0 && g == 0 && tid == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
+  if (err && tid == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
     const int r = r0 + warp * RPW + rr;

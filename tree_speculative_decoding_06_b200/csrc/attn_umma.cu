@@ -98,22 +98,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for the lean full-tile path (finite x <= 8): x = j + f with j = round(x),
-// found by adding 1.5 * 2^23 (j then sits in the low mantissa bits), and f in [-0.5, 0.5].  2^f
-// is a cubic whose coefficients were fitted here for least maximum relative error on that
-// interval (7.5e-5, well below the bf16 rounding that P gets before P V), and j is added to the
-// exponent field.  x below -125 is clamped there (2^-125 instead of a smaller number: no effect
-// on a row whose largest term is 2^0 or more).  The multi-function unit has 1/8 of the FMA
-// pipe's lanes, so taking some exponentials off it shortens the softmax (the split of work
-// between the two units follows "FlashAttention-4", which emulates part of exp2 in software on
-// Blackwell for the same reason).
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
 // Paired fp32 arithmetic of sm_100 (one instruction for two lanes of work) and the three-input
 // maximum: the lean full-tile softmax issues a third fewer instructions with them.
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -144,11 +128,6 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, f
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
-
-// Of each group of four exponentials in a full tile, this many are computed by poly_exp2.  Measured
-// on B200: 1 of 4 made the MUFU-heavy forest case 18% slower and 2 of 4 40% slower -- the softmax
-// warps are bound by instruction issue, not by the multi-function unit -- so it is 0 for now.
-constexpr int kPolyPerQuad = 0;
 
 __device__ __forceinline__ void abort_cta(const AttnArgs& a, int b, volatile int* s_abort) {
   if (*s_abort == 0) {
@@ -590,10 +569,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
             float x0, x1, x2, x3;
             fma2(x0, x1, __uint_as_float(s0[c]), __uint_as_float(s0[c + 1]), sl2, sl2, nmu, nmu);
             fma2(x2, x3, __uint_as_float(s1[c]), __uint_as_float(s1[c + 1]), sl2, sl2, nmu, nmu);
-            const float p0 = kPolyPerQuad >= 4 ? poly_exp2(x0) : fast_exp2(x0);
-            const float p1 = kPolyPerQuad >= 3 ? poly_exp2(x1) : fast_exp2(x1);
-            const float p2 = kPolyPerQuad >= 2 ? poly_exp2(x2) : fast_exp2(x2);
-            const float p3 = kPolyPerQuad >= 1 ? poly_exp2(x3) : fast_exp2(x3);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            const float p2 = fast_exp2(x2), p3 = fast_exp2(x3);
             add2(suma[0], suma[1], suma[0], suma[1], p0, p1);
             add2(suma[2], suma[3], suma[2], suma[3], p2, p3);
             pk[c / 2] = pack_bf16x2(p0, p1);
@@ -728,7 +705,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         }
         if (row_ok) *reinterpret_cast<float2*>(wml + (base + r) * 2) = make_float2(M, l);
       }
-      if (err && split == 0 && mt == 0 && g == 0 && tid == 128) flag_status(a.status, b, TSD_ERR_CAPACITY);
+      if (err && tid == 128) flag_status(a.status, b, TSD_ERR_CAPACITY);
     }
     if (u.stage) {
       // every thread copies staged rows out with coalesced 16-byte stores

@@ -71,14 +71,15 @@ __device__ __forceinline__ void merge(float& zm, double& s, float zm2, double s2
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) stats_kernel(const T* __restrict__ zp, const T* __restrict__ zq, int V,
-                                                         int K, Temp tc, int chunks, Stat* __restrict__ part) {
+                                                         int K, Temp tc, int chunks, Stat* __restrict__ part,
+                                                         int vec) {
   pdl_trigger();   // the scan reads inputs only; pdl_wait() comes before the partial is written
   const int c = blockIdx.x, r = blockIdx.y, b = blockIdx.z;
   const T* row = chain_row(zp, zq, K, V, b, r);
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
   float zm = -INFINITY;
   double s = 0.0;
-  if ((V & 7) == 0) {
+  if (vec) {
     for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
       float x[8];
       load8<T>(row, v, x);
@@ -373,10 +374,11 @@ tsd_status launch_chain_sample_stochastic(const void* zp, const void* zq, tsd_dt
   tc.lo = (float)(tc.c - (double)tc.hi);
   const size_t st_smem = (size_t)(2 * K + 1) * sizeof(Stat) + (size_t)2 * K * sizeof(float) + 16;
   dim3 g1(chunks, 2 * K + 1, B), g2(chunks, B);
+  const int vec = vec16_rows(zp, V) && (K == 0 || vec16_rows(zq, V)) ? 1 : 0;
   if (dtype == TSD_BF16) {
     auto p = reinterpret_cast<const __nv_bfloat16*>(zp);
     auto q = reinterpret_cast<const __nv_bfloat16*>(zq);
-    launch_pdl(stats_kernel<__nv_bfloat16>, g1, dim3(kThreads), 0, stream, p, q, V, K, tc, chunks, part);
+    launch_pdl(stats_kernel<__nv_bfloat16>, g1, dim3(kThreads), 0, stream, p, q, V, K, tc, chunks, part, vec);
     launch_pdl(mass_kernel<__nv_bfloat16>, g2, dim3(kThreads), st_smem, stream, p, q, x, u, V, K, tc, chunks,
                (const Stat*)part, mass, jbuf);
     launch_pdl(select_kernel<__nv_bfloat16>, dim3(B), dim3(kThreads), 0, stream, p, q, x, u, V, K, tc, chunks,
@@ -384,7 +386,7 @@ tsd_status launch_chain_sample_stochastic(const void* zp, const void* zq, tsd_dt
   } else {
     auto p = reinterpret_cast<const float*>(zp);
     auto q = reinterpret_cast<const float*>(zq);
-    launch_pdl(stats_kernel<float>, g1, dim3(kThreads), 0, stream, p, q, V, K, tc, chunks, part);
+    launch_pdl(stats_kernel<float>, g1, dim3(kThreads), 0, stream, p, q, V, K, tc, chunks, part, vec);
     launch_pdl(mass_kernel<float>, g2, dim3(kThreads), st_smem, stream, p, q, x, u, V, K, tc, chunks,
                (const Stat*)part, mass, jbuf);
     launch_pdl(select_kernel<float>, dim3(B), dim3(kThreads), 0, stream, p, q, x, u, V, K, tc, chunks, (const Stat*)part,

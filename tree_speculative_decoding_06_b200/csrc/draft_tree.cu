@@ -63,7 +63,7 @@ __device__ __forceinline__ void topk_at(const float (&tv)[kMaxK], const int (&ti
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict__ logits, int V, int F, int K,
-                                                            int chunks, uint8_t* __restrict__ ws) {
+                                                            int chunks, uint8_t* __restrict__ ws, int vec) {
   pdl_trigger();
   const int c = blockIdx.x, f = blockIdx.y, b = blockIdx.z;
   const T* row = logits + ((size_t)b * F + f) * V;
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
       topk_at(tv, ti, K - 1, thr_v, thr_i);
     }
   };
-  if ((V & 7) == 0) {
+  if (vec) {
     for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
       float x[8];
       load8<T>(row, v, x);
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
   // fp64 sum of fp32 exponentials relative to the chunk maximum (second pass, cache-resident)
   double sum = 0.0;
   if (M != -INFINITY) {
-    if ((V & 7) == 0) {
+    if (vec) {
       for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
         float x[8];
         load8<T>(row, v, x);
@@ -347,12 +347,13 @@ tsd_status launch_draft_expand(const DraftTreeArgs& t, const void* logits, tsd_d
   if (K < 1 || K > kMaxK || t.F < 1 || t.F > kMaxK || dt_chunks(V) > 64) return TSD_ERR_INVALID_ARG;
   const int chunks = dt_chunks(V);
   dim3 grid(chunks, t.F, t.B);
+  const int vec = vec16_rows(logits, V) ? 1 : 0;
   if (dtype == TSD_BF16)
     launch_pdl(draft_row_stats<__nv_bfloat16>, grid, dim3(kThreads), 0, stream,
-               reinterpret_cast<const __nv_bfloat16*>(logits), V, t.F, K, chunks, reinterpret_cast<uint8_t*>(ws));
+               reinterpret_cast<const __nv_bfloat16*>(logits), V, t.F, K, chunks, reinterpret_cast<uint8_t*>(ws), vec);
   else
     launch_pdl(draft_row_stats<float>, grid, dim3(kThreads), 0, stream, reinterpret_cast<const float*>(logits), V, t.F,
-               K, chunks, reinterpret_cast<uint8_t*>(ws));
+               K, chunks, reinterpret_cast<uint8_t*>(ws), vec);
   if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
   const size_t smem = (size_t)t.F * chunks * dt_rec_bytes(K);   // <= 16 x 64 x 144 B
   if (smem > 48 * 1024)

@@ -12,6 +12,15 @@
 
 namespace tsd {
 
+// The vocabulary scans read 8 logits (16 bytes of bf16, two 16-byte words of fp32) per load when
+// every row starts on a 16-byte boundary: V a multiple of 8 and the base pointer 16-byte aligned.
+// Decided on the host from the actual pointer, so a view at an odd storage offset takes the
+// scalar path instead of faulting.
+inline bool vec16_rows(const void* base, int V) {
+  return V % 8 == 0 && (reinterpret_cast<uintptr_t>(base) & 15) == 0;
+}
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 // Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger in common.cuh).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,

@@ -13,7 +13,13 @@ runs tsd_tree_accept_commit after the attention on one stream (and can splice th
 into a device token history); "serial" runs tsd_tree_accept_greedy then tsd_kv_commit on one
 stream.  A linear draft takes tsd_chain_accept_sample -> tsd_kv_commit[_paged] (length mode).
 
-and returns the device tensors it wrote.  The cache and prefix_len in `inputs` are updated in
+In the overlap schedule the acceptance reads status[b] while the attention may still be flagging
+that sequence (a bad block id, a capacity error, a timed-out wait): for a sequence whose status is
+non-zero after the step, accept_len / path / out_tokens are unspecified (the other schedules give
+the miss outputs).  The commit always reads the final status, so the status words, the caches and
+prefix_len come out the same under every schedule.
+
+run() returns the device tensors it wrote.  The cache and prefix_len in `inputs` are updated in
 place by the commit, exactly as a decoding loop would carry them into the next step; with
 history_cap > 0 the emitted tokens are also appended to a device token history.
 """
@@ -85,6 +91,10 @@ class VerifyStep:
         if self.accept == "greedy":
             return n + (2 if self.fused else 3)
         return n + (3 if self.T > 0 else 2) + 1
+
+    def attn_launches(self) -> int:
+        """Kernels one attention call launches (the split kernel, and its merge when split)."""
+        return 1 + int(self.splits_merge)
 
     def _accept(self, x: dict):
         tree_accept_greedy(x["logits"], x["tokens"], self.parent_s, x.get("num_nodes"), x.get("root_key"),
