@@ -265,6 +265,42 @@ tsd_status tsd_chain_accept_sample(const void *target_logits, const void *draft_
                                    size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------------------
+ * tsd_tree_accept_sample -- stochastic acceptance of a draft tree (temperature > 0)
+ * ([SO] "Objetivo-Borrador": accept a draft token with probability min(1, p/q), the rule of the
+ * cited Leviathan et al. paper, and sample one more token from the target after the accepted
+ * run; [SO] "EAGLE": the draft is a tree of candidates).  Reading for a tree whose children were
+ * drawn independently from their parent's draft distribution: starting at the root (node 0), the
+ * children of the current node are tried in index order; child c with token x is accepted iff
+ *   u[b,c] * q(x) < p(x),
+ * and after each rejection p is replaced by max(p - q, 0) / sum (kept when that sum is 0), so
+ * the next child is tested against the residual the earlier rejections left.  Acceptance moves
+ * to the accepted child and repeats; when no child is accepted (or the node is a leaf, or depth
+ * Dmax is reached) the last token is the smallest t with sum_{v<=t} p(v) > u[b,0] * sum_v p(v)
+ * for the current p.  p = softmax(target_logits[b,n] / T), q = softmax(draft_logits[b,n] / T)
+ * at node n.  With one child per node this is tsd_chain_accept_sample's rule.
+ *
+ *   target_logits [B, Nmax, V] dtype: row n = the target distribution after node n
+ *   draft_logits  [B, Nmax, V] dtype: row n = the draft distribution node n's children were drawn
+ *                 from (rows of leaves are not read)
+ *   tokens        [B, Nmax] int32; parent_s [B, Nmax+1] from tsd_tree_prepare (single-root trees:
+ *                 forest = 0)
+ *   uniforms      [B, Nmax] fp32 in [0,1): entry c (c >= 1) for the test of node c, entry 0 for
+ *                 the final draw
+ *   temperature   > 0 (use tsd_tree_accept_greedy for T = 0)
+ *   accept_len, path, out_tokens as in tsd_tree_accept_greedy (path = slots of the accepted nodes,
+ *                 out_tokens = the accepted drafts below the root, then the drawn token, -1 beyond)
+ *   status        [B] int32: a flagged sequence is skipped (accept_len -1); a node on the walk with
+ *                 more than 256 children flags TSD_ERR_INVALID_ARG (detail = that node)
+ * V is bounded by shared memory: 2 * ceil(V / 8) * sizeof(dtype) + 4 * Nmax <= 200 KiB.
+ * One launch (a cluster of 8 CTAs per sequence), no workspace.
+ * --------------------------------------------------------------------------------------- */
+tsd_status tsd_tree_accept_sample(const void *target_logits, const void *draft_logits, tsd_dtype dtype, int V,
+                                  const int32_t *tokens, const int32_t *parent_s, const int32_t *num_nodes,
+                                  const float *uniforms, float temperature, int B, int Nmax, int Dmax,
+                                  int32_t *accept_len, int32_t *path, int32_t *out_tokens, int32_t *status,
+                                  void *stream);
+
+/* ---------------------------------------------------------------------------------------
  * tsd_kv_commit -- commit the accepted path's K/V rows into the contiguous cache
  * ([EP] sec. 2, branchable KV cache: committed prefix state is kept apart from per-branch
  * speculative state; commit either keeps the first A steps (length) or follows the path

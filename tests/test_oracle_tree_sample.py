@@ -85,3 +85,25 @@ def test_special_cases():
     q2 = np.array([0, 0, 0.25, 0.25, 0.25, 0.25])
     path, em = ts.tree_accept_sample([-1, 0, 0], [0, 3, 5], [p2, p2, p2], [q2, q2, q2], [0.1, 0.1, 0.1, 0.7])
     assert path == [0] and em == [1]
+
+
+def test_batch_wrapper_marshals_the_gpu_layout():
+    """The batch form (GPU layout: uniforms[c] tests node c, uniforms[0] is the final draw, rows
+    of logits per node) gives what the single-tree form gives on the same trees and numbers, and
+    one margin per accept test plus one for the final draw."""
+    import workloads as W
+    parents = [W.tree_static_scored((4, 3, 2, 1, 1, 1), 26), W.tree_tiny(), W.tree_chain(4)]
+    inp = W.make_tree_sample_inputs(parents, 50, "f32", seed=4, T=0.8)
+    r = ts.tree_accept_sample_batch(inp["z_p"], inp["z_q"], inp["tokens"], inp["parent"], inp["num_nodes"],
+                                    inp["u"], 0.8, int(inp["Dmax"]), lambda row: np.asarray(row, np.float32))
+    for b, par in enumerate(parents):
+        N = len(par)
+        u = list(inp["u"][b, :N].astype(np.float64)) + [float(inp["u"][b, 0])]
+        P = [ts.softmax(inp["z_p"][b, i].astype(np.float64), 0.8) for i in range(N)]
+        Q = [ts.softmax(inp["z_q"][b, i].astype(np.float64), 0.8) for i in range(N)]
+        m = []
+        path, em = ts.tree_accept_sample([int(x) for x in par], [int(t) for t in inp["tokens"][b, :N]], P, Q, u, m)
+        assert r["accept_len"][b] == len(path) - 1
+        assert list(r["path"][b, :len(path)]) == [p + 1 for p in path] and (r["path"][b, len(path):] == 0).all()
+        assert list(r["out_tokens"][b, :len(em)]) == em and (r["out_tokens"][b, len(em):] == -1).all()
+        assert r["margins"][b] == m and len(m) >= 1

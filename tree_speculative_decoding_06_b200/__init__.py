@@ -46,6 +46,7 @@ _SIGS = {
     "tsd_tree_accept_greedy_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "tsd_tree_accept_greedy_noalloc_scratch_bytes": (_SZ, []),
     "tsd_chain_accept_sample_workspace_size": (_SZ, [_I, _I, _I]),
+    "tsd_tree_accept_sample": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _F, _I, _I, _I, _P, _P, _P, _P, _P]),
     "tsd_chain_accept_sample": (_I, [_P, _P, _I, _I, _P, _P, _F, _I, _I, _P, _P, _P, _SZ, _P]),
     "tsd_kv_commit": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "tsd_kv_commit_paged": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
@@ -287,6 +288,31 @@ def chain_accept_sample(target_logits, draft_logits, draft_tokens, uniforms, tem
                                        _stream(stream))
     _check(rc, "tsd_chain_accept_sample")
     return {"accept_len": accept_len, "out_tokens": out_tokens}
+
+
+def tree_accept_sample(target_logits, draft_logits, tokens, parent_s, uniforms, temperature: float,
+                       num_nodes=None, Dmax: int = 8, accept_len=None, path=None, out_tokens=None, status=None,
+                       stream=None):
+    """Stochastic acceptance of a draft tree (tsd_tree_accept_sample): target_logits / draft_logits
+    [B, N, V] (row n = after node n), tokens [B, N], uniforms [B, N] fp32 (entry c tests node c,
+    entry 0 is the final draw)."""
+    B, Nmax, V = target_logits.shape
+    if tuple(draft_logits.shape) != (B, Nmax, V) or draft_logits.dtype != target_logits.dtype:
+        raise TsdError("draft_logits must match target_logits in shape and dtype")
+    if uniforms.dtype != torch.float32 or tuple(uniforms.shape) != (B, Nmax):
+        raise TsdError("uniforms must be float32 [B, Nmax]")
+    accept_len = _empty((B,), torch.int32, target_logits) if accept_len is None else accept_len
+    path = _empty((B, Dmax + 1), torch.int32, target_logits) if path is None else path
+    out_tokens = _empty((B, Dmax + 1), torch.int32, target_logits) if out_tokens is None else out_tokens
+    if status is None:
+        status = torch.zeros(B, dtype=torch.int32, device=target_logits.device)
+    rc = lib().tsd_tree_accept_sample(_ptr(target_logits), _ptr(draft_logits), _dt(target_logits), V,
+                                      _i32(tokens, "tokens"), _i32(parent_s, "parent_s"),
+                                      _i32(num_nodes, "num_nodes"), _ptr(uniforms), float(temperature), B, Nmax,
+                                      Dmax, _ptr(accept_len), _ptr(path), _ptr(out_tokens), _ptr(status),
+                                      _stream(stream))
+    _check(rc, "tsd_tree_accept_sample")
+    return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
 
 
 # ----------------------------------------------------------------------------- commit

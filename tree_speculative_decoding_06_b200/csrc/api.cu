@@ -193,6 +193,23 @@ tsd_status tsd_chain_accept_sample(const void* target_logits, const void* draft_
                              accept_len, out_tokens, workspace, S(stream));
 }
 
+tsd_status tsd_tree_accept_sample(const void* target_logits, const void* draft_logits, tsd_dtype dtype, int V,
+                                  const int32_t* tokens, const int32_t* parent_s, const int32_t* num_nodes,
+                                  const float* uniforms, float temperature, int B, int Nmax, int Dmax,
+                                  int32_t* accept_len, int32_t* path, int32_t* out_tokens, int32_t* status,
+                                  void* stream) {
+  if (!dtype_ok(dtype)) return TSD_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || B > 65535 || Nmax < 0 || Nmax > 4096 || V <= 0 || Dmax < 0 || Dmax > 255) return TSD_ERR_INVALID_ARG;
+  if (!(temperature > 0.f) || !(temperature < 3.0e38f)) return TSD_ERR_INVALID_ARG;
+  if (tree_sample_smem(V, Nmax, dtype) > 200 * 1024) return TSD_ERR_INVALID_ARG;
+  if (B == 0) return TSD_OK;
+  if (!accept_len || !path || !out_tokens || !status || !parent_s || !uniforms ||
+      (Nmax > 0 && (!target_logits || !draft_logits || !tokens)))
+    return TSD_ERR_INVALID_ARG;
+  return launch_tree_sample(target_logits, draft_logits, dtype, V, tokens, parent_s, num_nodes, uniforms,
+                            temperature, B, Nmax, Dmax, accept_len, path, out_tokens, status, S(stream));
+}
+
 static tsd_status commit_common(CommitArgs& a, const void* k_tree, const void* v_tree, const int32_t* path,
                                 const int32_t* accept_len, tsd_dtype dtype, tsd_commit_mode mode) {
   if (!dtype_ok(dtype)) return TSD_ERR_UNSUPPORTED_DTYPE;

@@ -101,6 +101,13 @@ tsd_status launch_chain_sample(const void* zp, const void* zq, tsd_dtype dtype, 
                                const float* u, float T, int B, int K, int32_t* accept_len, int32_t* out_tokens,
                                void* ws, cudaStream_t stream);
 
+// Stochastic tree acceptance (tree_sample.cu): one cluster of CTAs per sequence.
+size_t tree_sample_smem(int V, int Nmax, tsd_dtype dtype);
+tsd_status launch_tree_sample(const void* zp, const void* zq, tsd_dtype dtype, int V, const int32_t* tokens,
+                              const int32_t* parent_s, const int32_t* num_nodes, const float* u, float T, int B,
+                              int Nmax, int Dmax, int32_t* accept_len, int32_t* path, int32_t* out_tokens,
+                              int32_t* status, cudaStream_t stream);
+
 struct CommitArgs {
   void* k_cache;
   void* v_cache;

@@ -463,3 +463,41 @@ def make_custom_inputs(parents, prefix_lens, Hq: int = 4, Hkv: int = 2, d: int =
                 tokens[b, i] = int(rng.integers(0, V))
     out.update(logits=logits, tokens=tokens, root_key=None)
     return out
+
+
+def make_tree_sample_inputs(parents, V: int, dtype: str = "bf16", seed: int = 0, T: float = 1.0,
+                            sigma: float = 2.0, noise: float = 0.8, Nmax: Optional[int] = None) -> dict:
+    """Inputs of stochastic tree acceptance for hand-picked trees (ragged, padded with -1 parents):
+    target logits z_p [B, Nmax, V] ~ N(0, sigma) per node row, draft logits z_q = z_p + N(0, noise)
+    (the chain workload's recipe), every non-root node's token drawn from softmax(z_q[parent] / T)
+    -- children of one node drawn independently, as the draft would -- the root's token uniform,
+    and uniforms u [B, Nmax] in [0, 1) (entry c for node c's test, entry 0 for the final draw)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    B = len(parents)
+    Ns = [len(p) for p in parents]
+    Nmax = max(Ns) if Nmax is None else Nmax
+    parent = np.full((B, Nmax), -1, np.int32)
+    for b, p in enumerate(parents):
+        parent[b, :len(p)] = p
+    store = np.uint16 if dtype == "bf16" else np.float32
+    zp = np.zeros((B, Nmax, V), store)
+    zq = np.zeros((B, Nmax, V), store)
+    tokens = np.zeros((B, Nmax), np.int32)
+    for b in range(B):
+        zpf = rng.standard_normal((Nmax, V), dtype=np.float32) * np.float32(sigma)
+        zqf = zpf + rng.standard_normal((Nmax, V), dtype=np.float32) * np.float32(noise)
+        zp[b] = f32_to_bf16_bits(zpf) if dtype == "bf16" else zpf
+        zq[b] = f32_to_bf16_bits(zqf) if dtype == "bf16" else zqf
+        tokens[b, 0] = rng.integers(0, V)
+        cdf = {}
+        for i in range(1, Ns[b]):
+            p = int(parent[b, i])
+            if p not in cdf:   # draft token drawn from softmax(z_q / T) (input construction)
+                z = as_f32(zq[b, p], dtype).astype(np.float64) / T
+                cdf[p] = np.cumsum(np.exp(z - z.max()))
+            c = cdf[p]
+            tokens[b, i] = min(int(np.searchsorted(c, rng.random() * c[-1], side="right")), V - 1)
+    u = rng.random((B, Nmax), dtype=np.float32)
+    Dmax = max(int(tree_depths(np.asarray(p)).max()) for p in parents)
+    return {"parent": parent, "num_nodes": np.asarray(Ns, np.int32), "z_p": zp, "z_q": zq, "tokens": tokens,
+            "u": u, "T": T, "Dmax": Dmax, "dtype": dtype}
