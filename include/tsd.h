@@ -301,6 +301,35 @@ tsd_status tsd_tree_accept_sample(const void *target_logits, const void *draft_l
                                   void *stream);
 
 /* ---------------------------------------------------------------------------------------
+ * tsd_ssd_cache_build -- the outcome cache of one SSD / Saguaro verification round
+ * ([SSD] sec. 2 and sec. 3 A-B: while the target verifies, the draft predicts the outcome --
+ * the accepted length and the bonus token -- and pre-drafts for the likely outcomes; the cache
+ * budget follows a geometric fan-out over the likely accepted lengths; Saguaro sampling lowers
+ * the draft probability of the cached tokens while drafting).  Reading of those passages:
+ *   P(a) = alpha^a (1 - alpha) for a < K, P(K) = alpha^K   (accepted length a of K drafts);
+ *   slots[b,a] = the largest-remainder apportionment of S slots in proportion to P(a)
+ *     (floor(S P(a)), then +1 to the largest remainders, ties -> shorter length);
+ *   the slots[b,a] outcome keys of length a are the most likely tokens of the draft distribution
+ *     at position a+1, q_a = softmax(draft_logits[b,a] / T) (ties -> lower id);
+ *   draft_tokens[b,j] (j < K) = the smallest t with sum_{v<=t} q'(v) > u[b,j] * sum_v q'(v),
+ *     q' = q_j * (beta on the keys of length j, 1 elsewhere), renormalised (q_j if that sum is 0).
+ *
+ *   draft_logits  [B, K+1, V] dtype: row a = the draft logits at position a+1 (row K: the free
+ *                 token after K accepted drafts; keys only)
+ *   alpha         [B] fp32 per-sequence acceptance rate (clamped to [0, 1])
+ *   beta          in [0, 1];  uniforms [B, K] fp32 in [0, 1);  temperature > 0
+ *   slots         [B, K+1] int32 out: slots per accepted length (sum S)
+ *   key_len, key_tok [B, S] int32 out: the outcome keys (accepted length, bonus token), ordered by
+ *                 length, then by draft probability (desc), then token id
+ *   draft_tokens  [B, K] int32 out
+ * Limits: 1 <= S <= 256, S <= V, 0 <= K <= 63, ceil(V / 8) * sizeof(dtype) <= 200 KiB.
+ * One launch (a cluster of 8 CTAs per (sequence, row)), no workspace.
+ * --------------------------------------------------------------------------------------- */
+tsd_status tsd_ssd_cache_build(const void *draft_logits, tsd_dtype dtype, int V, int K, int S, const float *alpha,
+                               float beta, const float *uniforms, float temperature, int B, int32_t *slots,
+                               int32_t *key_len, int32_t *key_tok, int32_t *draft_tokens, void *stream);
+
+/* ---------------------------------------------------------------------------------------
  * tsd_kv_commit -- commit the accepted path's K/V rows into the contiguous cache
  * ([EP] sec. 2, branchable KV cache: committed prefix state is kept apart from per-branch
  * speculative state; commit either keeps the first A steps (length) or follows the path

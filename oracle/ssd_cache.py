@@ -82,22 +82,31 @@ def saguaro_probs(logits: np.ndarray, cached, beta: float, T: float = 1.0) -> np
     return qp / s if s > 0 else q
 
 
-def inverse_cdf(prob: np.ndarray, u: float) -> int:
-    """Smallest t with sum_{v<=t} prob[v] > u * sum(prob) (sequential scan)."""
+def inverse_cdf(prob: np.ndarray, u: float, margin: list | None = None) -> int:
+    """Smallest t with sum_{v<=t} prob[v] > u * sum(prob) (sequential scan).  With `margin`,
+    appends the distance of the threshold to the nearest cumulative boundary of the chosen
+    token, relative to the total."""
     total = float(prob.sum())
     thr = u * total
     acc = 0.0
     for t, x in enumerate(prob):
+        prev = acc
         acc += float(x)
         if acc > thr:
+            if margin is not None:
+                margin.append(min(thr - prev, acc - thr) / total if total > 0 else 0.0)
             return t
+    if margin is not None:
+        margin.append(0.0)
     return int(np.nonzero(prob > 0)[0][-1])
 
 
-def build_and_draft(draft_logits: np.ndarray, S: int, alpha: float, beta: float, u: np.ndarray, T: float = 1.0):
+def build_and_draft(draft_logits: np.ndarray, S: int, alpha: float, beta: float, u: np.ndarray, T: float = 1.0,
+                    margins: list | None = None):
     """One sequence: fan-out, keys, and the K Saguaro-sampled draft tokens (u: K uniforms).
 
-    Returns dict(n, keys, tokens, probs) with probs[j] = q' of position j+1."""
+    Returns dict(n, keys, tokens, probs) with probs[j] = q' of position j+1; with `margins`,
+    appends each draw's margin (see inverse_cdf)."""
     K = draft_logits.shape[0] - 1
     n = geometric_fanout(S, alpha, K)
     keys = cache_keys(draft_logits, n, T)
@@ -106,5 +115,5 @@ def build_and_draft(draft_logits: np.ndarray, S: int, alpha: float, beta: float,
         cached = [t for a, t in keys if a == j]
         qp = saguaro_probs(draft_logits[j], cached, beta, T)
         probs.append(qp)
-        tokens.append(inverse_cdf(qp, float(u[j])))
+        tokens.append(inverse_cdf(qp, float(u[j]), margins))
     return {"n": n, "keys": keys, "tokens": np.array(tokens, np.int32), "probs": probs}

@@ -46,6 +46,7 @@ _SIGS = {
     "tsd_tree_accept_greedy_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "tsd_tree_accept_greedy_noalloc_scratch_bytes": (_SZ, []),
     "tsd_chain_accept_sample_workspace_size": (_SZ, [_I, _I, _I]),
+    "tsd_ssd_cache_build": (_I, [_P, _I, _I, _I, _I, _P, _F, _P, _F, _I, _P, _P, _P, _P, _P]),
     "tsd_tree_accept_sample": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _F, _I, _I, _I, _P, _P, _P, _P, _P]),
     "tsd_chain_accept_sample": (_I, [_P, _P, _I, _I, _P, _P, _F, _I, _I, _P, _P, _P, _SZ, _P]),
     "tsd_kv_commit": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -313,6 +314,25 @@ def tree_accept_sample(target_logits, draft_logits, tokens, parent_s, uniforms, 
                                       _stream(stream))
     _check(rc, "tsd_tree_accept_sample")
     return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
+
+
+def ssd_cache_build(draft_logits, alpha, beta: float, uniforms, S: int, temperature: float = 1.0, slots=None,
+                    key_len=None, key_tok=None, draft_tokens=None, stream=None):
+    """SSD / Saguaro outcome cache (tsd_ssd_cache_build): draft_logits [B, K+1, V], alpha [B] fp32,
+    uniforms [B, K] fp32.  Returns slots [B, K+1], key_len / key_tok [B, S], draft_tokens [B, K]."""
+    B, K1, V = draft_logits.shape
+    K = K1 - 1
+    if alpha.dtype != torch.float32 or uniforms.dtype != torch.float32:
+        raise TsdError("alpha and uniforms must be float32")
+    slots = _empty((B, K + 1), torch.int32, draft_logits) if slots is None else slots
+    key_len = _empty((B, S), torch.int32, draft_logits) if key_len is None else key_len
+    key_tok = _empty((B, S), torch.int32, draft_logits) if key_tok is None else key_tok
+    draft_tokens = _empty((B, max(K, 1)), torch.int32, draft_logits) if draft_tokens is None else draft_tokens
+    rc = lib().tsd_ssd_cache_build(_ptr(draft_logits), _dt(draft_logits), V, K, S, _ptr(alpha), float(beta),
+                                   _ptr(uniforms), float(temperature), B, _ptr(slots), _ptr(key_len), _ptr(key_tok),
+                                   _ptr(draft_tokens), _stream(stream))
+    _check(rc, "tsd_ssd_cache_build")
+    return {"slots": slots, "key_len": key_len, "key_tok": key_tok, "draft_tokens": draft_tokens}
 
 
 # ----------------------------------------------------------------------------- commit

@@ -210,6 +210,21 @@ tsd_status tsd_tree_accept_sample(const void* target_logits, const void* draft_l
                             temperature, B, Nmax, Dmax, accept_len, path, out_tokens, status, S(stream));
 }
 
+tsd_status tsd_ssd_cache_build(const void* draft_logits, tsd_dtype dtype, int V, int K, int S, const float* alpha,
+                               float beta, const float* uniforms, float temperature, int B, int32_t* slots,
+                               int32_t* key_len, int32_t* key_tok, int32_t* draft_tokens, void* stream) {
+  if (!dtype_ok(dtype)) return TSD_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || B > 65535 || V <= 0 || K < 0 || K > ssd_cache_max_k() || S < 1 || S > ssd_cache_max_slots() || S > V)
+    return TSD_ERR_INVALID_ARG;
+  if (!(beta >= 0.f && beta <= 1.f) || !(temperature > 0.f) || !(temperature < 3.0e38f)) return TSD_ERR_INVALID_ARG;
+  if (ssd_cache_smem(V, dtype) > 200 * 1024) return TSD_ERR_INVALID_ARG;
+  if (B == 0) return TSD_OK;
+  if (!draft_logits || !alpha || !slots || !key_len || !key_tok || (K > 0 && (!uniforms || !draft_tokens)))
+    return TSD_ERR_INVALID_ARG;
+  return launch_ssd_cache(draft_logits, dtype, V, K, S, alpha, beta, uniforms, temperature, B, slots, key_len,
+                          key_tok, draft_tokens, ::S(stream));
+}
+
 static tsd_status commit_common(CommitArgs& a, const void* k_tree, const void* v_tree, const int32_t* path,
                                 const int32_t* accept_len, tsd_dtype dtype, tsd_commit_mode mode) {
   if (!dtype_ok(dtype)) return TSD_ERR_UNSUPPORTED_DTYPE;

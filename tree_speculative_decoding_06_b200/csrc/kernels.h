@@ -108,6 +108,14 @@ tsd_status launch_tree_sample(const void* zp, const void* zq, tsd_dtype dtype, i
                               int Nmax, int Dmax, int32_t* accept_len, int32_t* path, int32_t* out_tokens,
                               int32_t* status, cudaStream_t stream);
 
+// SSD / Saguaro outcome cache (ssd_cache.cu): one cluster of CTAs per (sequence, row).
+size_t ssd_cache_smem(int V, tsd_dtype dtype);
+int ssd_cache_max_slots();
+int ssd_cache_max_k();
+tsd_status launch_ssd_cache(const void* zq, tsd_dtype dtype, int V, int K, int S, const float* alpha, float beta,
+                            const float* u, float T, int B, int32_t* slots, int32_t* key_len, int32_t* key_tok,
+                            int32_t* draft_tokens, cudaStream_t stream);
+
 struct CommitArgs {
   void* k_cache;
   void* v_cache;

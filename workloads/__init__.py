@@ -501,3 +501,15 @@ def make_tree_sample_inputs(parents, V: int, dtype: str = "bf16", seed: int = 0,
     Dmax = max(int(tree_depths(np.asarray(p)).max()) for p in parents)
     return {"parent": parent, "num_nodes": np.asarray(Ns, np.int32), "z_p": zp, "z_q": zq, "tokens": tokens,
             "u": u, "T": T, "Dmax": Dmax, "dtype": dtype}
+
+
+def make_ssd_inputs(B: int, K: int, V: int, dtype: str = "bf16", seed: int = 0, sigma: float = 3.0,
+                    alpha_lo: float = 0.4, alpha_hi: float = 0.9) -> dict:
+    """Inputs of the SSD outcome-cache build: draft logits [B, K+1, V] ~ N(0, sigma) (row a = the
+    draft distribution at position a+1), a per-sequence acceptance rate alpha ~ U[alpha_lo,
+    alpha_hi] (fp32) and uniforms [B, K] in [0, 1) (fp32) for the K draft draws."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    z = _normal(rng, (B, K + 1, V), sigma, dtype)
+    alpha = rng.uniform(alpha_lo, alpha_hi, size=B).astype(np.float32)
+    u = rng.random((B, K), dtype=np.float32)
+    return {"draft_logits": z, "alpha": alpha, "u": u, "dtype": dtype, "K": K, "V": V}
