@@ -585,6 +585,22 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
   p.tps = best_tps;
   p.splits = (p.max_tiles + p.tps - 1) / p.tps;
   if (p.splits < 1) p.splits = 1;
+  // tcgen05 kernel: the CTAs splitting one row block's keys form a cluster and merge their
+  // partials through distributed shared memory, so a split costs no extra memory traffic or
+  // launch; each takes an equal share of its own sequence's tiles (ragged lengths stay balanced
+  // inside a cluster).  Fill the machine first (at least one CTA per SM when the row blocks alone
+  // do not), then minimise waves * (tiles per CTA + overhead) at the capacity length.
+  if (umma_shape) {
+    const long long ubase = (long long)B * Hkv * p.umtiles;
+    int cmin = ubase >= sms ? 1 : (int)((sms + ubase - 1) / ubase);
+    if (cmin > 16) cmin = 16;
+    double best = 1e300;
+    for (int c = cmin; c <= 16; ++c) {
+      const double waves = (double)((ubase * c + sms - 1) / sms);
+      const double cost = waves * ((p.max_tiles + c - 1) / c + overhead);
+      if (cost < best - 1e-9) best = cost, p.csize = c;
+    }
+  }
   p.ws_bytes = p.splits > 1 ? (size_t)B * Hkv * p.splits * p.Rmax * (d + 2) * sizeof(float) : 0;
   return p;
 }
@@ -597,8 +613,7 @@ tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t str
   const char* path_env = getenv("TSD_ATTN_PATH");
   const bool force_mma = path_env != nullptr && path_env[0] == 'm' && path_env[1] == 'm';
   if (dtype == TSD_BF16 && !force_mma && umma_eligible(a, dtype)) {
-    const tsd_status st = launch_attention_umma(a, p, stream);
-    if (st != TSD_OK) return st;
+    return launch_attention_umma(a, p, stream);   // splits merge inside their cluster
   } else if (dtype == TSD_BF16) {
     if (a.d == 128) {
       set_smem_attr(attn_bf16_kernel<128>, p.smem);

@@ -14,6 +14,7 @@ namespace attn {
 struct SeqView {
   int N, R, L, nPT, T, nsplit;
   bool skip, zero;   // skip: nothing to do; zero: write zeros (flagged / out of capacity)
+  bool cap;          // out of capacity (decided by the inputs alone, unlike the status word)
 };
 
 __device__ __forceinline__ SeqView seq_view(const AttnArgs& a, int b, int G, int BN, int tps) {
@@ -24,6 +25,7 @@ __device__ __forceinline__ SeqView seq_view(const AttnArgs& a, int b, int G, int
   v.L = a.prefix_len[b];
   const bool in_cache = (a.k_tree == nullptr);
   const bool cap_bad = (v.L < 0) || ((long long)v.L + (in_cache ? v.N : 0) > a.Lcap);
+  v.cap = cap_bad;
   v.zero = cap_bad || (a.status[b] != 0);
   v.nPT = cap_bad ? 0 : (v.L + BN - 1) / BN;
   v.T = v.nPT + (v.N + BN - 1) / BN;

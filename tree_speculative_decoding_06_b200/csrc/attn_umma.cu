@@ -33,16 +33,20 @@
 //     16-byte stores.
 // Every mbarrier wait is bounded: on time-out the CTA records TSD_ERR_TIMEOUT, drains its own
 // TMA copies (again bounded) and frees its TMEM before returning.
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <climits>
+#include <cstdlib>
 #include <mutex>
 
 #include "attn_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "umma.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace tsd {
 
@@ -72,7 +76,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;               // lazy max: rescale only past a 2^8 growth
 
 struct UParams {
-  int tps, splits, Rmax, mtiles;
+  int csize;           // CTAs per (sequence, KV head, query-row block): a cluster splitting the keys
+  int mtiles;
+  long long wait;      // cycles after which an mbarrier wait gives up (TSD_ERR_TIMEOUT)
+  int withhold;        // test hook: the K producer never issues this tile (-1: off)
   int ks, vs;          // K and V ring depths
   int box_rows;        // rows per TMA box of the cache (64 contiguous, min(block, 64) paged)
   int W;               // ancestor-bit words per node
@@ -207,25 +214,33 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   __shared__ volatile int s_abort;
   __shared__ int s_k_issued, s_v_issued, s_k_consumed, s_v_consumed;
   __shared__ float2 s_ml1[kBM];   // warpgroup 1's (max, sum) per row, for the epilogue merge
+  constexpr int kRows = kDual ? 2 * kBM : kBM;   // query rows of this CTA
+  __shared__ float2 s_mlc[kRows];  // cluster split: this CTA's (max, sum) per row
+  __shared__ int s_bad;            // cluster split: this CTA's partial is unusable (time-out, bad block)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int mt = blockIdx.x % u.mtiles, split = blockIdx.x / u.mtiles;
+  // the CTAs of one (sequence, KV head, row block) are adjacent in x and form one cluster when
+  // csize > 1: CTA `split` takes an equal share of the sequence's key tiles
+  const int split = blockIdx.x % u.csize, mt = blockIdx.x / u.csize;
   const int g = blockIdx.y, b = blockIdx.z;
   const int G = a.Hq / a.Hkv;
-  const SeqView v = seq_view(a, b, G, kBN, u.tps);
-  constexpr int kRows = kDual ? 2 * kBM : kBM;   // query rows of this CTA
+  const SeqView v = seq_view(a, b, G, kBN, 1 << 30);
   const int r0 = mt * kRows;
+  // Every early return below is taken by all CTAs of a cluster alike: they share b, g, mt and
+  // decide from the inputs alone.  The status word is not such an input (another launch may flag
+  // the sequence while this one starts), so a clustered CTA only notes what it read and the
+  // cluster merge zeroes the rows if any CTA saw a flag.
   if (v.skip || r0 >= v.R) return;
   const int r_hi = min(r0 + kRows, v.R);
-  if (v.zero) {
+  const bool direct = (u.csize == 1);
+  if (direct ? v.zero : v.cap) {
     if (split == 0) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
     if (split == 0 && mt == 0 && g == 0 && tid == 0 && a.status[b] == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
     return;
   }
-  if (split >= v.nsplit) return;
-  const bool direct = (v.nsplit == 1);
-  const int t_begin = split * u.tps;
-  const int nt = min(v.T, t_begin + u.tps) - t_begin;
+  const bool entry_flag = !direct && v.zero;   // flagged before this launch
+  const int t_begin = (int)((long long)split * v.T / u.csize);
+  const int nt = (int)((long long)(split + 1) * v.T / u.csize) - t_begin;   // may be 0 when T < csize
   const int nodes_per_tile = kRows / G;
   const int node0 = mt * nodes_per_tile;
 
@@ -275,10 +290,11 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       TileBlocks nxt;
       fetch_blocks(a, v, u, b, t_begin, nxt);
       for (int i = 0; i < nt && !s_abort; ++i) {
+        if (t_begin + i == u.withhold) break;   // test hook: this tile never arrives
         const TileBlocks cur = nxt;
         if (i + 1 < nt) fetch_blocks(a, v, u, b, t_begin + i + 1, nxt);
         const int st = i % u.ks;
-        if (i >= u.ks && !mbar_wait(&bars.k_empty[st], ((i / u.ks) - 1) & 1)) {
+        if (i >= u.ks && !mbar_wait(&bars.k_empty[st], ((i / u.ks) - 1) & 1, u.wait)) {
           abort_cta(a, b, &s_abort);
           break;
         }
@@ -307,7 +323,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         const TileBlocks cur = nxt;
         if (i + 1 < nt) fetch_blocks(a, v, u, b, t_begin + i + 1, nxt);
         const int st = i % u.vs;
-        if (i >= u.vs && !mbar_wait(&bars.v_empty[st], ((i / u.vs) - 1) & 1)) {
+        if (i >= u.vs && !mbar_wait(&bars.v_empty[st], ((i / u.vs) - 1) & 1, u.wait)) {
           abort_cta(a, b, &s_abort);
           break;
         }
@@ -329,7 +345,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     // every lane waits and the verdict is made warp-uniform: the MMA issue below is
     // warp-collective (elect.sync) and needs the whole warp converged
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, u.wait)) != 0;
     };
     bool ok = wait_all(&bars.q_full, 0);
     int k_consumed = 0, v_consumed = 0;
@@ -492,7 +508,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       const int k = kDual ? i : i >> 1;            // this warpgroup's k-th tile
       const int buf = kDual ? wg : wg + 2 * (k & 1);
       const uint32_t s_col = kColS + (uint32_t)buf * kBN;
-      if (!mbar_wait(&bars.s_full[buf], kDual ? (k & 1) : ((k >> 1) & 1))) {
+      if (!mbar_wait(&bars.s_full[buf], kDual ? (k & 1) : ((k >> 1) & 1), u.wait)) {
         ok = false;
         break;
       }
@@ -523,7 +539,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           const int lim = tree ? v.N : v.L;
           uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
           if (tree && !mask_ready) {
-            if (!mbar_wait(&bars.mask_full, 0)) {
+            if (!mbar_wait(&bars.mask_full, 0, u.wait)) {
               ok = false;
               break;
             }
@@ -592,7 +608,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         l = l * alpha + ((suma[0] + suma[1]) + (suma[2] + suma[3]));
       }
       // this warpgroup's previous P V (tile i - 2) must be done before O is rescaled
-      if (k >= 1 && !mbar_wait(&bars.pv_done[wg], (k - 1) & 1)) {
+      if (k >= 1 && !mbar_wait(&bars.pv_done[wg], (k - 1) & 1, u.wait)) {
         ok = false;
         break;
       }
@@ -619,7 +635,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     }
     // the warpgroup's last P V product
     const int kn = kDual ? nt : (nt - wg + 1) >> 1;   // tiles this warpgroup processed
-    if (ok && kn > 0 && !mbar_wait(&bars.pv_done[wg], (kn - 1) & 1)) ok = false;
+    if (ok && kn > 0 && !mbar_wait(&bars.pv_done[wg], (kn - 1) & 1, u.wait)) ok = false;
     if (!ok) abort_cta(a, b, &s_abort);
     row_m = m_used;
     row_l = l;
@@ -680,10 +696,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         if (row_ok && a.lse)
           a.lse[((size_t)b * a.Nmax + i_node) * a.Hq + g * G + hh] = err ? 0.f : (M + __log2f(l)) * kLn2;
       } else {
-        // split-KV partial: unnormalised O relative to M, with (M, l)
-        float* wo = reinterpret_cast<float*>(a.workspace);
-        const size_t base = (((size_t)b * a.Hkv + g) * u.splits + split) * u.Rmax;
-        float* wml = wo + (size_t)a.B * a.Hkv * u.splits * u.Rmax * kD;
+        // cluster split: this CTA's partial row (unnormalised O relative to M, and (M, l)) stays in
+        // its own shared memory, where the cluster's merge reads it
 #pragma unroll
         for (int ch = 0; ch < kD / 32; ++ch) {
           uint32_t o0[32], o1[32];
@@ -691,8 +705,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           if (two) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
           tmem_wait_ld();
           if (row_ok) {
-            float4* dst = u.stage ? reinterpret_cast<float4*>(sStage + (size_t)crow * kStageF + ch * 128)
-                                  : reinterpret_cast<float4*>(wo + (base + r) * kD + ch * 32);
+            float4* dst = reinterpret_cast<float4*>(sStage + (size_t)crow * kStageF + ch * 128);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               float f[4];
@@ -703,42 +716,73 @@ __global__ void __launch_bounds__(kThreadsU, 1)
             }
           }
         }
-        if (row_ok) *reinterpret_cast<float2*>(wml + (base + r) * 2) = make_float2(M, l);
+        s_mlc[crow] = make_float2(l > 0.f ? M : -INFINITY, l);
       }
       if (err && tid == 128) flag_status(a.status, b, TSD_ERR_CAPACITY);
     }
-    if (u.stage) {
+    if (u.stage && direct) {
       // every thread copies staged rows out with coalesced 16-byte stores
       __syncthreads();
       const int nrows = r_hi - r0;
-      if (direct) {
-        for (int idx = tid; idx < nrows * (kD / 8); idx += kThreadsU) {
-          const int cr = idx / (kD / 8), c = idx % (kD / 8);
-          const int rr = r0 + cr, node = rr / G, hh = rr % G;
-          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
-                                (((size_t)b * a.Nmax + node) * a.Hq + g * G + hh) * kD;
-          reinterpret_cast<uint4*>(orow)[c] = *reinterpret_cast<const uint4*>(sStage + (size_t)cr * kStageH + c * 16);
-        }
-      } else {
-        float* wo = reinterpret_cast<float*>(a.workspace);
-        const size_t base = (((size_t)b * a.Hkv + g) * u.splits + split) * u.Rmax + r0;
-        for (int idx = tid; idx < nrows * (kD / 4); idx += kThreadsU) {
-          const int cr = idx / (kD / 4), c = idx % (kD / 4);
-          reinterpret_cast<float4*>(wo + (base + cr) * kD)[c] =
-              *reinterpret_cast<const float4*>(sStage + (size_t)cr * kStageF + c * 16);
-        }
+      for (int idx = tid; idx < nrows * (kD / 8); idx += kThreadsU) {
+        const int cr = idx / (kD / 8), c = idx % (kD / 8);
+        const int rr = r0 + cr, node = rr / G, hh = rr % G;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
+                              (((size_t)b * a.Nmax + node) * a.Hq + g * G + hh) * kD;
+        reinterpret_cast<uint4*>(orow)[c] = *reinterpret_cast<const uint4*>(sStage + (size_t)cr * kStageH + c * 16);
       }
     }
   } else {
     // time-out: let this CTA's own TMA copies and MMAs land (bounded) before freeing TMEM
     if (tid == 0) {
-      for (int i = s_k_consumed; i < s_k_issued; ++i) mbar_wait(&bars.k_full[i % u.ks], (i / u.ks) & 1);
-      for (int i = s_v_consumed; i < s_v_issued; ++i) mbar_wait(&bars.v_full[i % u.vs], (i / u.vs) & 1);
+      for (int i = s_k_consumed; i < s_k_issued; ++i) mbar_wait(&bars.k_full[i % u.ks], (i / u.ks) & 1, u.wait);
+      for (int i = s_v_consumed; i < s_v_issued; ++i) mbar_wait(&bars.v_full[i % u.vs], (i / u.vs) & 1, u.wait);
     }
     if (warp == 3 && lane == 0) {
       tc_commit(&bars.fin);
-      mbar_wait(&bars.fin, 0);
+      mbar_wait(&bars.fin, 0, u.wait);
     }
+    for (int i = tid; i < kRows; i += kThreadsU) s_mlc[i] = make_float2(-INFINITY, 0.f);
+    if (direct) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
+  }
+  if (!direct) {
+    // ------------------------------------------------------------ cluster merge of the split partials
+    // Each CTA of the cluster merges an equal share of the rows: for row r, with partials
+    // (O_s, M_s, l_s) of the cluster's CTAs s, out = sum_s 2^(M_s - M) O_s / sum_s 2^(M_s - M) l_s,
+    // M = max_s M_s, read from the peers' shared memory (distributed shared memory).  Two cluster
+    // barriers: partials complete before any read, reads complete before any CTA leaves.  Every CTA
+    // reaches both (all waits above are bounded).
+    cg::cluster_group cl = cg::this_cluster();
+    if (tid == 0) s_bad = (s_abort || s_err || entry_flag) ? 1 : 0;
+    __syncthreads();
+    cl.sync();
+    int anybad = 0;
+    for (int s2 = 0; s2 < u.csize; ++s2) anybad |= *cl.map_shared_rank(&s_bad, s2);
+    const int nrows = r_hi - r0;
+    const int q_lo = (int)((long long)split * nrows / u.csize);
+    const int q_hi = (int)((long long)(split + 1) * nrows / u.csize);
+    for (int crow = q_lo + warp; crow < q_hi; crow += kThreadsU / 32) {
+      float2 ml = make_float2(-INFINITY, 0.f);
+      if (lane < u.csize) ml = *cl.map_shared_rank(&s_mlc[crow], lane);
+      const float M = warp_max(ml.x);
+      const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+      const float L = warp_sum(ml.y * w);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s2 = 0; s2 < u.csize; ++s2) {
+        const float ws = __shfl_sync(0xffffffffu, w, s2);
+        if (ws == 0.f) continue;   // an empty or unusable partial (its rows may hold anything)
+        const float4 x = cl.map_shared_rank(reinterpret_cast<const float4*>(sStage + (size_t)crow * kStageF), s2)[lane];
+        acc.x = fmaf(x.x, ws, acc.x), acc.y = fmaf(x.y, ws, acc.y);
+        acc.z = fmaf(x.z, ws, acc.z), acc.w = fmaf(x.w, ws, acc.w);
+      }
+      const float inv = (L > 0.f && !anybad) ? 1.f / L : 0.f;
+      const int rr = r0 + crow, node = rr / G, hh = rr % G;
+      const size_t orow = (((size_t)b * a.Nmax + node) * a.Hq + g * G + hh);
+      reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + orow * kD)[lane] =
+          make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+      if (a.lse && lane == 0) a.lse[orow] = (L > 0.f && !anybad) ? (M + __log2f(L)) * kLn2 : 0.f;
+    }
+    cl.sync();
   }
   tc_fence_before();
   __syncthreads();
@@ -788,10 +832,62 @@ bool umma_eligible(const AttnArgs& a, tsd_dtype dtype) {
   return encoder() != nullptr;
 }
 
+// Largest cluster size <= want (halving) whose clusters the device can hold at least one of with
+// this kernel and shared-memory size; sizes above 8 need the non-portable opt-in.  Answers are
+// cached per (kernel, size, shared memory).
+int cluster_fit(const void* kernel, int want, size_t smem, int mtiles, int Hkv, int B) {
+  static std::mutex mu;
+  struct Key {
+    const void* k;
+    int c;
+    size_t s;
+    bool ok;
+  };
+  static Key memo[64];
+  static int nmemo = 0;
+  while (want > 1) {
+    bool ok = false, found = false;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      for (int i = 0; i < nmemo; ++i)
+        if (memo[i].k == kernel && memo[i].c == want && memo[i].s == smem) ok = memo[i].ok, found = true;
+    }
+    if (!found) {
+      if (want > 8) cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(mtiles * want, Hkv, B);
+      cfg.blockDim = dim3(kThreadsU);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = want, attr[0].val.clusterDim.y = 1, attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      ok = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n >= 1;
+      cudaGetLastError();
+      std::lock_guard<std::mutex> lock(mu);
+      if (nmemo < 64) memo[nmemo++] = Key{kernel, want, smem, ok};
+    }
+    if (ok) return want;
+    want = want > 8 ? 8 : want / 2;
+  }
+  return 1;
+}
+
 tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   UParams u{};
-  u.tps = p.tps, u.splits = p.splits, u.Rmax = p.Rmax, u.mtiles = p.umtiles;
+  u.csize = p.csize, u.mtiles = p.umtiles;
+  u.wait = kWaitCycles;
+  u.withhold = -1;
+  // Test hook for the bounded waits: TSD_TEST_WITHHOLD_TILE=t makes the K producer of every CTA
+  // skip key tile t (and every later one), so the waits on it give up after 10^5 cycles and the
+  // call reports TSD_ERR_TIMEOUT in status[] instead of stalling.
+  if (const char* w = getenv("TSD_TEST_WITHHOLD_TILE")) {
+    u.withhold = atoi(w);
+    u.wait = 100000;
+  }
   const int rows = p.dual ? 2 * kBM : kBM;   // query rows per CTA
   const uint32_t q_bytes = p.dual ? 0u : kQBytes;   // two query tiles live in TMEM, not shared memory
   u.W = (a.Nmax + 31) / 32;
@@ -801,7 +897,7 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
     return 1024 + q_bytes + (uint32_t)(ks + vs) * kSlot + ((mask_bytes + 15) & ~15u) + ps_bytes;
   };
   u.ks = 6, u.vs = 5;   // K is consumed first (by S = Q K^T), so its ring runs further ahead
-  const uint32_t limit = 227 * 1024 - 2048;   // leave room for the static shared variables
+  const uint32_t limit = 227 * 1024 - 4096;   // leave room for the static shared variables
   while (total(u.ks, u.vs) > limit && u.vs > 2) {
     if (u.ks > u.vs) --u.ks; else --u.vs;
   }
@@ -845,9 +941,21 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   }
   auto kernel = p.dual ? attn_umma_kernel<true> : attn_umma_kernel<false>;
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  dim3 grid(u.mtiles * p.splits, a.Hkv, a.B);
-  if (launch_pdl(kernel, grid, dim3(kThreadsU), smem, stream, mq, mk, mv, mkt, mvt, a, u) != cudaSuccess)
-    return TSD_ERR_CUDA;
+  if (!u.stage) u.csize = 1;   // the cluster merge stages partial rows in the idle K/V rings
+  u.csize = cluster_fit(reinterpret_cast<const void*>(kernel), u.csize, smem, u.mtiles, a.Hkv, a.B);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(u.mtiles * u.csize, a.Hkv, a.B);
+  cfg.blockDim = dim3(kThreadsU);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = u.csize, attr[1].val.clusterDim.y = 1, attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = u.csize > 1 ? 2 : 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, mkt, mvt, a, u) != cudaSuccess) return TSD_ERR_CUDA;
   return TSD_OK;
 }
 

@@ -49,7 +49,8 @@ struct AttnPlan {
   int max_tiles = 0;        // prefix tiles at capacity + tree tiles
   int tps = 1, splits = 1;  // tiles per split, splits per (sequence, KV head, row tile)
   bool dual = false;        // tcgen05 kernel: two 128-row query tiles per CTA
-  int umtiles = 0;          // tcgen05 kernel: CTAs per (sequence, KV head, split)
+  int umtiles = 0;          // tcgen05 kernel: row blocks per (sequence, KV head)
+  int csize = 1;            // tcgen05 kernel: CTAs (one cluster) splitting the keys of a row block
   int threads = 128;
   size_t smem = 0;
   size_t ws_bytes = 0;
