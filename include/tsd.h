@@ -207,6 +207,29 @@ tsd_status tsd_tree_accept_greedy(const void *logits, tsd_dtype dtype, int V, co
                                   void *stream);
 
 /* ---------------------------------------------------------------------------------------
+ * tsd_tree_accept_threshold -- threshold acceptance over the tree
+ * ([SO] "Decodificacion especulativa": besides exact matching, the target may keep the longest
+ * prefix whose tokens stay above an acceptance threshold; the page gives no formula).  Reading:
+ * with p_n = softmax(logits[b,n] / T), a non-root node i is accepted iff its parent is accepted
+ * and p_parent(i)(tokens[b,i]) >= tau (fp64 comparison); roots, the deepest-node rule, the path
+ * and the emitted tokens (the last one = argmax of the deepest accepted node's row) are exactly
+ * those of tsd_tree_accept_greedy.  tau = 0 accepts every node; tau > 1/2 accepts only argmax
+ * tokens.
+ *
+ *   logits, tokens, parent_s, num_nodes, root_key, outputs, status: as tsd_tree_accept_greedy
+ *   tau           threshold in [0, 1];  temperature > 0
+ *   workspace     >= tsd_tree_accept_threshold_workspace_size(B, Nmax, V) bytes
+ * Two launches (the vocabulary scan, then one CTA per sequence); Nmax <= 4096.
+ * --------------------------------------------------------------------------------------- */
+size_t tsd_tree_accept_threshold_workspace_size(int B, int Nmax, int V);
+
+tsd_status tsd_tree_accept_threshold(const void *logits, tsd_dtype dtype, int V, const int32_t *tokens,
+                                     const int32_t *parent_s, const int32_t *num_nodes, const int32_t *root_key,
+                                     float tau, float temperature, int B, int Nmax, int Dmax,
+                                     int32_t *accept_len, int32_t *path, int32_t *out_tokens, void *workspace,
+                                     size_t ws_bytes, int32_t *status, void *stream);
+
+/* ---------------------------------------------------------------------------------------
  * tsd_tree_accept_greedy_noalloc -- tsd_tree_accept_greedy for callers that cannot allocate.
  * The pages have no counterpart of this call; it exists for library users whose code may not
  * call cudaMalloc: a serving engine that gave all free device memory to its KV-cache pool at

@@ -354,7 +354,8 @@ def _bits(t):
 
 
 @pytest.mark.parametrize("name,schedule", [(n, s) for n in ("tiny", "tree26", "eagle60", "forest")
-                                            for s in ("overlap", "fused", "serial")] + [("chain5", None)])
+                                            for s in ("overlap", "fused", "serial")] +
+                         [("chain5", "overlap"), ("chain5", "serial")])
 def test_verify_step_matches_oracle(name, schedule):
     """The whole step under each schedule: the attention output of every row within tolerance,
     acceptance bit-exact (margin protocol for sampling), and the K and V caches byte-exact after

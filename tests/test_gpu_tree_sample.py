@@ -90,7 +90,7 @@ def test_tree_sample_matches_oracle(V, dt):
 
 def test_tree_sample_full_size_eagle2_trees():
     """B = 16 EAGLE-2 trees of 60 nodes over the 128256-token vocabulary (bf16)."""
-    w = W.WORKLOADS["eagle60"].scaled(L=16)
+    w = W.WORKLOADS["eagle60"].scaled(L=16, L_lo=8)
     base = W.make_inputs(w, nan_guard=False)
     parents = [base["parent"][b, :int(base["num_nodes"][b])] for b in range(w.B)]
     inp = W.make_tree_sample_inputs(parents, 128256, "bf16", seed=5, T=1.0)

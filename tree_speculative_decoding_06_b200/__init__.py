@@ -43,6 +43,8 @@ _SIGS = {
                                         _I, _F, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_accept_greedy_workspace_size": (_SZ, [_I, _I, _I]),
     "tsd_tree_accept_greedy": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
+    "tsd_tree_accept_threshold_workspace_size": (_SZ, [_I, _I, _I]),
+    "tsd_tree_accept_threshold": (_I, [_P, _I, _I, _P, _P, _P, _P, _F, _F, _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_accept_greedy_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "tsd_tree_accept_greedy_noalloc_scratch_bytes": (_SZ, []),
     "tsd_chain_accept_sample_workspace_size": (_SZ, [_I, _I, _I]),
@@ -241,6 +243,32 @@ def tree_accept_greedy(logits, tokens, parent_s, num_nodes=None, root_key=None, 
                                       _i32(root_key, "root_key"), B, Nmax, Dmax, _ptr(accept_len), _ptr(path),
                                       _ptr(out_tokens), _ptr(workspace), nbytes, _ptr(status), _stream(stream))
     _check(rc, "tsd_tree_accept_greedy")
+    return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
+
+
+def tree_accept_threshold_workspace_size(B, Nmax, V) -> int:
+    return int(lib().tsd_tree_accept_threshold_workspace_size(B, Nmax, V))
+
+
+def tree_accept_threshold(logits, tokens, parent_s, tau: float, temperature: float = 1.0, num_nodes=None,
+                          root_key=None, Dmax: int = 8, accept_len=None, path=None, out_tokens=None, workspace=None,
+                          status=None, stream=None):
+    """Threshold acceptance over the tree (tsd_tree_accept_threshold): a node is accepted while its
+    parent's target distribution gives its token probability >= tau."""
+    B, Nmax, V = logits.shape
+    accept_len = _empty((B,), torch.int32, logits) if accept_len is None else accept_len
+    path = _empty((B, Dmax + 1), torch.int32, logits) if path is None else path
+    out_tokens = _empty((B, Dmax + 1), torch.int32, logits) if out_tokens is None else out_tokens
+    if status is None:
+        status = torch.zeros(B, dtype=torch.int32, device=logits.device)
+    nbytes = tree_accept_threshold_workspace_size(B, Nmax, V)
+    workspace = _ws(nbytes, logits, workspace)
+    rc = lib().tsd_tree_accept_threshold(_ptr(logits), _dt(logits), V, _i32(tokens, "tokens"),
+                                         _i32(parent_s, "parent_s"), _i32(num_nodes, "num_nodes"),
+                                         _i32(root_key, "root_key"), float(tau), float(temperature), B, Nmax, Dmax,
+                                         _ptr(accept_len), _ptr(path), _ptr(out_tokens), _ptr(workspace), nbytes,
+                                         _ptr(status), _stream(stream))
+    _check(rc, "tsd_tree_accept_threshold")
     return {"accept_len": accept_len, "path": path, "out_tokens": out_tokens}
 
 

@@ -48,7 +48,9 @@ __device__ __forceinline__ void merge_rows_warp(const float2* s_part, int chunks
   }
 }
 
-// Acceptance of sequence b by the whole CTA.  s_tstar holds >= Nmax ints of shared memory;
+// Acceptance of sequence b by the whole CTA.  s_tstar holds >= Nmax ints of shared memory
+// (already filled when tstar_ready); match, if not null, holds one byte per node: edge
+// parent(i) -> i passes iff match[i] != 0, instead of the greedy token test;
 // s_stage, if not null, >= 2 * Nmax + 1 more, into which the tree's parent slots and tokens are
 // copied first (one coalesced read each) so that the ancestor walks run on shared memory;
 // s_part, if not null, holds Nmax * chunks float2: every row's argmax partials are read into it
@@ -65,7 +67,8 @@ __device__ __forceinline__ int tree_accept_block(const float2* __restrict__ part
                                                  const int32_t* __restrict__ status, int32_t* __restrict__ accept_len,
                                                  int32_t* __restrict__ path, int32_t* __restrict__ out_tokens,
                                                  int32_t* s_tstar, int32_t* s_path, int32_t* s_stage,
-                                                 float2* s_part) {
+                                                 float2* s_part, const uint8_t* match = nullptr,
+                                                 bool tstar_ready = false) {
   __shared__ int s_hit, s_best, s_A;
   const int b = blockIdx.x;
   const int N = num_nodes ? num_nodes[b] : Nmax;
@@ -83,7 +86,9 @@ __device__ __forceinline__ int tree_accept_block(const float2* __restrict__ part
     tok = s_stage + Nmax + 1;
   }
   if (threadIdx.x == 0) s_hit = INT_MAX, s_best = -1;
-  if (s_part != nullptr) {
+  if (tstar_ready) {
+    // the caller filled s_tstar[0..N) (visible after the __syncthreads below)
+  } else if (s_part != nullptr) {
     const float2* src = part + (size_t)b * Nmax * chunks;
     for (int k = threadIdx.x; k < Nmax * chunks; k += blockDim.x) s_part[k] = src[k];
     __syncthreads();
@@ -118,7 +123,9 @@ __device__ __forceinline__ int tree_accept_block(const float2* __restrict__ part
         ok = false;
         break;
       }
-      ok = ok && (tok[s - 1] == s_tstar[p - 1]);
+      // greedy: the token is the parent's argmax; with a match table (threshold acceptance) the
+      // caller decided every edge
+      ok = ok && (match ? match[s - 1] != 0 : tok[s - 1] == s_tstar[p - 1]);
       s = p;
       ++d;
       if (!ok) break;

@@ -151,6 +151,28 @@ tsd_status tsd_tree_accept_greedy(const void* logits, tsd_dtype dtype, int V, co
                               path, out_tokens, workspace, status, S(stream));
 }
 
+size_t tsd_tree_accept_threshold_workspace_size(int B, int Nmax, int V) {
+  if (B <= 0 || Nmax <= 0 || V <= 0) return 0;
+  return accept_threshold_ws(B, Nmax, V);
+}
+
+tsd_status tsd_tree_accept_threshold(const void* logits, tsd_dtype dtype, int V, const int32_t* tokens,
+                                     const int32_t* parent_s, const int32_t* num_nodes, const int32_t* root_key,
+                                     float tau, float temperature, int B, int Nmax, int Dmax, int32_t* accept_len,
+                                     int32_t* path, int32_t* out_tokens, void* workspace, size_t ws_bytes,
+                                     int32_t* status, void* stream) {
+  if (!dtype_ok(dtype)) return TSD_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || B > 65535 || Nmax < 0 || Nmax > 4096 || V <= 0 || Dmax < 0 || Dmax > 255) return TSD_ERR_INVALID_ARG;
+  if (!(tau >= 0.f && tau <= 1.f) || !(temperature > 0.f) || !(temperature < 3.0e38f)) return TSD_ERR_INVALID_ARG;
+  if (B == 0) return TSD_OK;
+  if (!accept_len || !path || !out_tokens || !status || !parent_s || (Nmax > 0 && (!logits || !tokens)))
+    return TSD_ERR_INVALID_ARG;
+  const size_t need = tsd_tree_accept_threshold_workspace_size(B, Nmax, V);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace))) return TSD_ERR_WORKSPACE;
+  return launch_accept_threshold(logits, dtype, V, tokens, parent_s, num_nodes, root_key, tau, temperature, B, Nmax,
+                                 Dmax, accept_len, path, out_tokens, workspace, status, S(stream));
+}
+
 tsd_status tsd_tree_accept_greedy_noalloc(const void* logits, tsd_dtype dtype, int V, const int32_t* tokens,
                                           const int32_t* parent_s, const int32_t* num_nodes,
                                           const int32_t* root_key, int B, int Nmax, int Dmax,

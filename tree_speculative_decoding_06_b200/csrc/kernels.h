@@ -117,6 +117,15 @@ tsd_status launch_ssd_cache(const void* zq, tsd_dtype dtype, int V, int K, int S
                             const float* u, float T, int B, int32_t* slots, int32_t* key_len, int32_t* key_tok,
                             int32_t* draft_tokens, cudaStream_t stream);
 
+// Threshold acceptance (accept_threshold.cu).
+size_t accept_threshold_ws(int B, int Nmax, int V);
+size_t accept_threshold_smem(int Nmax);
+tsd_status launch_accept_threshold(const void* logits, tsd_dtype dtype, int V, const int32_t* tokens,
+                                   const int32_t* parent_s, const int32_t* num_nodes, const int32_t* root_key,
+                                   float tau, float T, int B, int Nmax, int Dmax, int32_t* accept_len,
+                                   int32_t* path, int32_t* out_tokens, void* ws, int32_t* status,
+                                   cudaStream_t stream);
+
 struct CommitArgs {
   void* k_cache;
   void* v_cache;

@@ -5,13 +5,14 @@ enqueues, on the current stream and without any host synchronisation,
 
     tsd_tree_prepare -> tsd_tree_verify_attn[_paged] -> acceptance -> tsd_kv_commit[_paged]
 
-The greedy acceptance depends on the tree and the target logits only, not on the attention, so by
-default (schedule "overlap") it runs on a second stream forked after prepare -- the vocabulary scan
-and the acceptance then use the SMs the attention leaves idle -- and the commit (which must follow
-the attention: it advances prefix_len, which the attention reads) joins both.  Schedule "fused"
+The acceptance (greedy, or the chain sampler) depends on the tree and the logits only, not on the
+attention, so by default (schedule "overlap") it runs on a second stream forked after prepare --
+the vocabulary scans and the decisions then use the SMs and memory cycles the attention leaves
+idle -- and the commit (which must follow the attention: it advances prefix_len, which the
+attention reads) joins both.  Schedule "fused"
 runs tsd_tree_accept_commit after the attention on one stream (and can splice the emitted tokens
-into a device token history); "serial" runs tsd_tree_accept_greedy then tsd_kv_commit on one
-stream.  A linear draft takes tsd_chain_accept_sample -> tsd_kv_commit[_paged] (length mode).
+into a device token history); "serial" runs the acceptance then tsd_kv_commit on one stream.  A
+linear draft takes tsd_chain_accept_sample -> tsd_kv_commit[_paged] (length mode).
 
 In the overlap schedule the acceptance reads status[b] while the attention may still be flagging
 that sequence (a bad block id, a capacity error, a timed-out wait): for a sequence whose status is
@@ -41,12 +42,12 @@ class VerifyStep:
                  schedule: Optional[str] = None, history_cap: int = 0, T: float = 0.0, device="cuda"):
         self.B, self.Nmax, self.Hq, self.Hkv, self.d, self.Dmax, self.V = B, Nmax, Hq, Hkv, d, Dmax, V
         self.dtype, self.paged, self.forest, self.accept, self.K = dtype, paged, forest, accept, K
-        if accept != "greedy":
-            schedule = "serial"
-        elif schedule is None:
-            schedule = "fused" if history_cap > 0 else "overlap"
+        if schedule is None:
+            schedule = "fused" if history_cap > 0 and accept == "greedy" else "overlap"
         if schedule not in ("overlap", "fused", "serial"):
             raise ValueError(f"unknown schedule {schedule!r}")
+        if schedule == "fused" and accept != "greedy":
+            raise ValueError("the fused schedule is greedy acceptance + commit")
         if history_cap > 0 and schedule != "fused":
             raise ValueError("a token history needs the fused schedule")
         self.schedule = schedule
@@ -101,9 +102,13 @@ class VerifyStep:
         return 1 + int(self.splits_merge)
 
     def _accept(self, x: dict):
-        tree_accept_greedy(x["logits"], x["tokens"], self.parent_s, x.get("num_nodes"), x.get("root_key"),
-                           self.Dmax, accept_len=self.accept_len, path=self.path, out_tokens=self.out_tokens,
-                           workspace=self.acc_ws, status=self.status)
+        if self.accept == "greedy":
+            tree_accept_greedy(x["logits"], x["tokens"], self.parent_s, x.get("num_nodes"), x.get("root_key"),
+                               self.Dmax, accept_len=self.accept_len, path=self.path, out_tokens=self.out_tokens,
+                               workspace=self.acc_ws, status=self.status)
+        else:
+            chain_accept_sample(x["z_p"], x["z_q"], x["x"], x["u"], x["T"], accept_len=self.accept_len,
+                                out_tokens=self.out_tokens, workspace=self.acc_ws)
 
     def run(self, x: dict) -> dict:
         tree_prepare(x["parent"], x.get("num_nodes"), self.Dmax, self.forest, parent_s=self.parent_s,
@@ -135,16 +140,11 @@ class VerifyStep:
                                workspace=self.acc_ws, status=self.status)
             return {"out": self.out, "accept_len": self.accept_len, "path": self.path,
                     "out_tokens": self.out_tokens, "status": self.status, "parent_s": self.parent_s}
-        if self.accept == "greedy":
-            if self.schedule == "overlap":
-                main.wait_event(self.ev_join)
-            else:
-                self._accept(x)
-            mode = "path"
+        if self.schedule == "overlap":
+            main.wait_event(self.ev_join)
         else:
-            chain_accept_sample(x["z_p"], x["z_q"], x["x"], x["u"], x["T"], accept_len=self.accept_len,
-                                out_tokens=self.out_tokens, workspace=self.acc_ws)
-            mode = "length"
+            self._accept(x)
+        mode = "path" if self.accept == "greedy" else "length"
         if self.paged:
             kv_commit_paged(x["k_pages"], x["v_pages"], x["block_table"], x["prefix_len"], x["k_tree"], x["v_tree"],
                             self.path, self.accept_len, x.get("num_nodes"), self.Dmax, mode, status=self.status)
