@@ -62,10 +62,11 @@ def test_host_argument_checks():
 
 
 def test_workspace_sizes_are_consistent():
-    # the paged query equals the contiguous one at the same capacity
+    # the paged query plans for ragged lengths (more splits), so it never asks for less than the
+    # contiguous one at the same capacity; both cover the partials of every split the plan makes
     a = tsd.tree_verify_attn_workspace_size(16, 60, 32, 8, 128, 8320, 1)
     b = tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1)
-    assert a == b
+    assert b >= a and b % (16 * 8 * 240 * 130 * 4) == 0
     assert tsd.tree_accept_greedy_workspace_size(8, 512, 128256) == 8 * 512 * 16 * 8
     assert tsd.chain_accept_sample_workspace_size(64, 5, 128256) > 64 * 11 * 16 * 8
 
@@ -100,12 +101,13 @@ def test_host_checks_of_the_fused_and_draft_tree_entry_points():
 
 def test_split_planner_choices_for_the_bench_workloads():
     """The planner's split counts (read back through the workspace size: splits * rows * (d + 2)
-    fp32 per KV head and sequence) for the four bench shapes on a 148-SM device; a split-count sweep
-    on B200 measured these as the fastest for tree26 (3..17) and eagle60 (1..4)."""
+    fp32 per KV head and sequence) for the four bench shapes on a 148-SM device: tree26 9 (a sweep
+    of 3..17 on B200 found 9 fastest), eagle60 3 (paged: planned for ragged lengths, each split an
+    equal share of its own sequence, longest sequences first), chain5 2, forest 2."""
     def splits(ws, B, Hkv, R, d=128):
         return ws // (B * Hkv * R * (d + 2) * 4) if ws else 1
     assert splits(tsd.tree_verify_attn_workspace_size(1, 26, 32, 8, 128, 2112, 1), 1, 8, 104) == 9
-    assert splits(tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1), 16, 8, 240) == 1
+    assert splits(tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1), 16, 8, 240) == 3
     assert splits(tsd.tree_verify_attn_workspace_size(64, 6, 64, 8, 128, 8256, 1), 64, 8, 48) == 2
     assert splits(tsd.tree_verify_attn_paged_workspace_size(8, 512, 32, 8, 128, 2080, 16, 1), 8, 8, 2048) == 2
 

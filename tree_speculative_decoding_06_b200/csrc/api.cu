@@ -70,13 +70,14 @@ tsd_status tsd_tree_prepare(const int32_t* parent, const int32_t* num_nodes, int
 
 size_t tsd_tree_verify_attn_workspace_size(int B, int Nmax, int Hq, int Hkv, int d, int Lmax, tsd_dtype dtype) {
   if (B <= 0 || Nmax <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Lmax < 0 || !dtype_ok(dtype)) return 0;
-  return plan_attention(B, Nmax, Hq, Hkv, d, Lmax, dtype).ws_bytes;
+  return plan_attention(B, Nmax, Hq, Hkv, d, Lmax, dtype, false).ws_bytes;
 }
 
 size_t tsd_tree_verify_attn_paged_workspace_size(int B, int Nmax, int Hq, int Hkv, int d, int max_blocks,
                                                  int block_size, tsd_dtype dtype) {
   if (max_blocks < 0 || block_size <= 0) return 0;
-  return tsd_tree_verify_attn_workspace_size(B, Nmax, Hq, Hkv, d, max_blocks * block_size, dtype);
+  if (B <= 0 || Nmax <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !dtype_ok(dtype)) return 0;
+  return plan_attention(B, Nmax, Hq, Hkv, d, max_blocks * block_size, dtype, true).ws_bytes;
 }
 
 tsd_status tsd_tree_verify_attn(const void* q, const void* k_cache, const void* v_cache, int Lmax,

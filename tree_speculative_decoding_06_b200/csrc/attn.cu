@@ -433,15 +433,19 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a, int BM,
 // ------------------------------------------------------------------------------------------
 constexpr int kFastSplits = 16;   // merges of up to this many splits load everything at once
 
+// equal != 0: every sequence has `splits` partials (the tcgen05 kernel's equal shares, where a
+// split with no keys wrote M = -inf); else ceil(tiles / tps) of them.  A partial whose weight is 0
+// is skipped without reading its O.
 template <int D, typename OutT>
-__global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int splits, int Rmax) {
+__global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int splits, int Rmax, int equal) {
   pdl_trigger();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * (blockDim.x >> 5) + warp;
   const int g = blockIdx.y, b = blockIdx.z;
   const int G = a.Hq / a.Hkv;
-  const SeqView v = seq_view(a, b, G, BN, tps);
+  SeqView v = seq_view(a, b, G, BN, tps);
+  if (equal) v.nsplit = splits;
   if (v.skip || r >= v.R) return;
   const int i = r / G, hh = r % G;
   OutT* orow = reinterpret_cast<OutT*>(a.out) + (((size_t)b * a.Nmax + i) * a.Hq + g * G + hh) * D;
@@ -461,16 +465,18 @@ __global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int split
     // columns of every split's partial row), so the merge waits for one round trip to memory
     float2 ml = make_float2(-INFINITY, 0.f);
     if (lane < v.nsplit) ml = *reinterpret_cast<const float2*>(wml + (base + (size_t)lane * Rmax) * 2);
+    const bool use = ml.x != -INFINITY;   // lanes >= nsplit hold (-inf, 0) too
+    const unsigned live = __ballot_sync(0xffffffffu, use);
     float ov[kFastSplits][D / 32];
 #pragma unroll
     for (int s = 0; s < kFastSplits; ++s) {
       const float* src = wo + (base + (size_t)s * Rmax) * D + lane;
 #pragma unroll
-      for (int e = 0; e < D / 32; ++e) ov[s][e] = s < v.nsplit ? src[32 * e] : 0.f;
+      for (int e = 0; e < D / 32; ++e) ov[s][e] = (live >> s) & 1u ? src[32 * e] : 0.f;
     }
     const float M = warp_max(ml.x);
     const float Mu = M == -INFINITY ? 0.f : M;
-    const float w = lane < v.nsplit ? exp2f(ml.x - Mu) : 0.f;
+    const float w = use ? exp2f(ml.x - Mu) : 0.f;
     const float lsum = warp_sum(ml.y * w);
     float acc[D / 32];
 #pragma unroll
@@ -503,13 +509,14 @@ __global__ void attn_combine_kernel(const AttnArgs a, int BN, int tps, int split
     float w = 0.f;
     if (s < v.nsplit) {
       const float2 ml = *reinterpret_cast<const float2*>(wml + (base + (size_t)s * Rmax) * 2);
-      w = exp2f(ml.x - Mu);
+      w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - Mu);
       lsum += ml.y * w;
     }
     const int n = min(32, v.nsplit - s0);
 #pragma unroll 4
     for (int k = 0; k < n; ++k) {
       const float wk = __shfl_sync(0xffffffffu, w, k);
+      if (wk == 0.f) continue;
       const float* src = wo + (base + (size_t)(s0 + k) * Rmax) * D + lane;
 #pragma unroll
       for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(src[32 * e], wk, acc[e]);
@@ -536,7 +543,7 @@ int device_sm_count() {
   return n > 0 ? n : 148;
 }
 
-AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype) {
+AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype, bool paged) {
   AttnPlan p;
   p.G = Hq / Hkv;
   p.Rmax = p.G * Nmax;
@@ -585,35 +592,47 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
   p.tps = best_tps;
   p.splits = (p.max_tiles + p.tps - 1) / p.tps;
   if (p.splits < 1) p.splits = 1;
-  // tcgen05 kernel: the CTAs splitting one row block's keys form a cluster and merge their
-  // partials through distributed shared memory, so a split costs no extra memory traffic or
-  // launch; each takes an equal share of its own sequence's tiles (ragged lengths stay balanced
-  // inside a cluster).  Fill the machine first (at least one CTA per SM when the row blocks alone
-  // do not), then minimise waves * (tiles per CTA + overhead) at the capacity length.
+  // tcgen05 kernel: CTA s of a row block's `usplits` takes the equal share [s T / n, (s+1) T / n)
+  // of its own sequence's T tiles and sequences are taken longest first, so a ragged batch stays
+  // balanced.  The host does not see the lengths: contiguous caches are costed at the capacity
+  // length (waves x tiles per CTA); paged caches, whose sequences are usually ragged, by the mean
+  // of that and a spread-lengths model (half the capacity on average: the larger of the longest
+  // CTA and the total work over the SMs).  Each split adds partials to write and merge.
   if (umma_shape) {
     const long long ubase = (long long)B * Hkv * p.umtiles;
-    int cmin = ubase >= sms ? 1 : (int)((sms + ubase - 1) / ubase);
-    if (cmin > 16) cmin = 16;
     double best = 1e300;
-    for (int c = cmin; c <= 16; ++c) {
+    for (int c = 1; c <= 32; ++c) {
+      const double per = (double)((p.max_tiles + c - 1) / c) + overhead;
       const double waves = (double)((ubase * c + sms - 1) / sms);
-      const double cost = waves * ((p.max_tiles + c - 1) / c + overhead);
-      if (cost < best - 1e-9) best = cost, p.csize = c;
+      double cost = waves * per;
+      if (paged) {
+        const double spread = fmax(per, (double)ubase * (0.5 * p.max_tiles + c * overhead) / sms);
+        cost = 0.5 * (cost + spread);
+      }
+      cost += c > 1 ? 0.35 * c : 0.0;
+      if (cost < best - 1e-9) best = cost, p.usplits = c;
     }
   }
-  p.ws_bytes = p.splits > 1 ? (size_t)B * Hkv * p.splits * p.Rmax * (d + 2) * sizeof(float) : 0;
+  const int wsplits = p.splits > p.usplits ? p.splits : p.usplits;   // either kernel may run
+  p.ws_bytes = wsplits > 1 ? (size_t)B * Hkv * wsplits * p.Rmax * (d + 2) * sizeof(float) : 0;
   return p;
 }
 
 tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream) {
   if (a.B == 0 || a.Nmax == 0) return TSD_OK;
-  const AttnPlan p = plan_attention(a.B, a.Nmax, a.Hq, a.Hkv, a.d, a.Lcap, dtype);
+  const AttnPlan p = plan_attention(a.B, a.Nmax, a.Hq, a.Hkv, a.d, a.Lcap, dtype, a.block_table != nullptr);
   dim3 grid(p.mtiles * p.splits, a.Hkv, a.B);
   // TSD_ATTN_PATH=mma selects the warp-level kernel even where the tcgen05 kernel applies (A/B runs)
   const char* path_env = getenv("TSD_ATTN_PATH");
   const bool force_mma = path_env != nullptr && path_env[0] == 'm' && path_env[1] == 'm';
   if (dtype == TSD_BF16 && !force_mma && umma_eligible(a, dtype)) {
-    return launch_attention_umma(a, p, stream);   // splits merge inside their cluster
+    const tsd_status st = launch_attention_umma(a, p, stream);
+    if (st != TSD_OK || p.usplits <= 1) return st;
+    const int rows_per_block = 8;
+    dim3 cg((p.Rmax + rows_per_block - 1) / rows_per_block, a.Hkv, a.B);
+    launch_pdl(attn_combine_kernel<128, __nv_bfloat16>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.usplits, p.Rmax,
+               1);
+    return cudaGetLastError() == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
   } else if (dtype == TSD_BF16) {
     if (a.d == 128) {
       set_smem_attr(attn_bf16_kernel<128>, p.smem);
@@ -637,14 +656,14 @@ tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t str
     dim3 cg((p.Rmax + rows_per_block - 1) / rows_per_block, a.Hkv, a.B);
     if (dtype == TSD_BF16) {
       if (a.d == 128)
-        launch_pdl(attn_combine_kernel<128, __nv_bfloat16>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax);
+        launch_pdl(attn_combine_kernel<128, __nv_bfloat16>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax, 0);
       else
-        launch_pdl(attn_combine_kernel<64, __nv_bfloat16>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax);
+        launch_pdl(attn_combine_kernel<64, __nv_bfloat16>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax, 0);
     } else {
       if (a.d == 128)
-        launch_pdl(attn_combine_kernel<128, float>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax);
+        launch_pdl(attn_combine_kernel<128, float>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax, 0);
       else
-        launch_pdl(attn_combine_kernel<64, float>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax);
+        launch_pdl(attn_combine_kernel<64, float>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.splits, p.Rmax, 0);
     }
     if (cudaGetLastError() != cudaSuccess) return TSD_ERR_CUDA;
   }

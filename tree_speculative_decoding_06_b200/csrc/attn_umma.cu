@@ -33,7 +33,6 @@
 //     16-byte stores.
 // Every mbarrier wait is bounded: on time-out the CTA records TSD_ERR_TIMEOUT, drains its own
 // TMA copies (again bounded) and frees its TMEM before returning.
-#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -45,8 +44,6 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "umma.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace tsd {
 
@@ -76,10 +73,12 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;               // lazy max: rescale only past a 2^8 growth
 
 struct UParams {
-  int csize;           // CTAs per (sequence, KV head, query-row block): a cluster splitting the keys
+  int splits;          // CTAs splitting one (sequence, KV head, row block)'s keys, equal shares
+  int Rmax;            // query rows per (sequence, KV head): the partials' row stride
   int mtiles;
   long long wait;      // cycles after which an mbarrier wait gives up (TSD_ERR_TIMEOUT)
   int withhold;        // test hook: the K producer never issues this tile (-1: off)
+  int lpt;             // map blockIdx.z to sequences by decreasing prefix length (B <= threads)
   int ks, vs;          // K and V ring depths
   int box_rows;        // rows per TMA box of the cache (64 contiguous, min(block, 64) paged)
   int W;               // ancestor-bit words per node
@@ -215,32 +214,46 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   __shared__ int s_k_issued, s_v_issued, s_k_consumed, s_v_consumed;
   __shared__ float2 s_ml1[kBM];   // warpgroup 1's (max, sum) per row, for the epilogue merge
   constexpr int kRows = kDual ? 2 * kBM : kBM;   // query rows of this CTA
-  __shared__ float2 s_mlc[kRows];  // cluster split: this CTA's (max, sum) per row
-  __shared__ int s_bad;            // cluster split: this CTA's partial is unusable (time-out, bad block)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // the CTAs of one (sequence, KV head, row block) are adjacent in x and form one cluster when
-  // csize > 1: CTA `split` takes an equal share of the sequence's key tiles
-  const int split = blockIdx.x % u.csize, mt = blockIdx.x / u.csize;
-  const int g = blockIdx.y, b = blockIdx.z;
+  // CTA `split` of a (sequence, KV head, row block) takes an equal share of that sequence's own key
+  // tiles (so ragged lengths stay balanced across its splits)
+  const int split = blockIdx.x % u.splits, mt = blockIdx.x / u.splits;
+  const int g = blockIdx.y;
+  // Sequences are taken longest prefix first (ties by index): blocks start in z order, so the
+  // longest sequences' CTAs start in the first wave and a ragged batch does not end on one long
+  // sequence.  Every CTA ranks the prefix lengths itself.
+  int b = blockIdx.z;
+  if (u.lpt) {
+    __shared__ int s_b;
+    if (tid < a.B) {
+      const int L = a.prefix_len[tid];
+      int rank = 0;
+      for (int o = 0; o < a.B; ++o) {
+        const int Lo = a.prefix_len[o];
+        rank += (Lo > L) || (Lo == L && o < tid);
+      }
+      if (rank == (int)blockIdx.z) s_b = tid;
+    }
+    __syncthreads();
+    b = s_b;
+  }
   const int G = a.Hq / a.Hkv;
   const SeqView v = seq_view(a, b, G, kBN, 1 << 30);
   const int r0 = mt * kRows;
-  // Every early return below is taken by all CTAs of a cluster alike: they share b, g, mt and
-  // decide from the inputs alone.  The status word is not such an input (another launch may flag
-  // the sequence while this one starts), so a clustered CTA only notes what it read and the
-  // cluster merge zeroes the rows if any CTA saw a flag.
   if (v.skip || r0 >= v.R) return;
   const int r_hi = min(r0 + kRows, v.R);
-  const bool direct = (u.csize == 1);
-  if (direct ? v.zero : v.cap) {
+  // a flagged or over-capacity sequence: zero rows (the split merge zeroes them too, as it reads
+  // the status after every split has finished)
+  if (v.zero) {
     if (split == 0) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
-    if (split == 0 && mt == 0 && g == 0 && tid == 0 && a.status[b] == 0) flag_status(a.status, b, TSD_ERR_CAPACITY);
+    if (split == 0 && mt == 0 && g == 0 && tid == 0 && a.status[b] == 0 && v.cap)
+      flag_status(a.status, b, TSD_ERR_CAPACITY);
     return;
   }
-  const bool entry_flag = !direct && v.zero;   // flagged before this launch
-  const int t_begin = (int)((long long)split * v.T / u.csize);
-  const int nt = (int)((long long)(split + 1) * v.T / u.csize) - t_begin;   // may be 0 when T < csize
+  const bool direct = (u.splits == 1);
+  const int t_begin = (int)((long long)split * v.T / u.splits);
+  const int nt = (int)((long long)(split + 1) * v.T / u.splits) - t_begin;   // 0 when T < splits
   const int nodes_per_tile = kRows / G;
   const int node0 = mt * nodes_per_tile;
 
@@ -696,8 +709,11 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         if (row_ok && a.lse)
           a.lse[((size_t)b * a.Nmax + i_node) * a.Hq + g * G + hh] = err ? 0.f : (M + __log2f(l)) * kLn2;
       } else {
-        // cluster split: this CTA's partial row (unnormalised O relative to M, and (M, l)) stays in
-        // its own shared memory, where the cluster's merge reads it
+        // split partial: unnormalised O relative to M, with (M, l); a split with no keys (or no
+        // mass) writes M = -inf, which the merge skips without reading its O
+        float* wo = reinterpret_cast<float*>(a.workspace);
+        const size_t base = (((size_t)b * a.Hkv + g) * u.splits + split) * u.Rmax;
+        float* wml = wo + (size_t)a.B * a.Hkv * u.splits * u.Rmax * kD;
 #pragma unroll
         for (int ch = 0; ch < kD / 32; ++ch) {
           uint32_t o0[32], o1[32];
@@ -705,7 +721,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           if (two) tmem_ld32(lane_addr + kColO + kD + ch * 32, o1);
           tmem_wait_ld();
           if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(sStage + (size_t)crow * kStageF + ch * 128);
+            float4* dst = u.stage ? reinterpret_cast<float4*>(sStage + (size_t)crow * kStageF + ch * 128)
+                                  : reinterpret_cast<float4*>(wo + (base + r) * kD + ch * 32);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               float f[4];
@@ -716,20 +733,30 @@ __global__ void __launch_bounds__(kThreadsU, 1)
             }
           }
         }
-        s_mlc[crow] = make_float2(l > 0.f ? M : -INFINITY, l);
+        if (row_ok) *reinterpret_cast<float2*>(wml + (base + r) * 2) = make_float2(l > 0.f ? M : -INFINITY, l);
       }
       if (err && tid == 128) flag_status(a.status, b, TSD_ERR_CAPACITY);
     }
-    if (u.stage && direct) {
+    if (u.stage) {
       // every thread copies staged rows out with coalesced 16-byte stores
       __syncthreads();
       const int nrows = r_hi - r0;
-      for (int idx = tid; idx < nrows * (kD / 8); idx += kThreadsU) {
-        const int cr = idx / (kD / 8), c = idx % (kD / 8);
-        const int rr = r0 + cr, node = rr / G, hh = rr % G;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
-                              (((size_t)b * a.Nmax + node) * a.Hq + g * G + hh) * kD;
-        reinterpret_cast<uint4*>(orow)[c] = *reinterpret_cast<const uint4*>(sStage + (size_t)cr * kStageH + c * 16);
+      if (direct) {
+        for (int idx = tid; idx < nrows * (kD / 8); idx += kThreadsU) {
+          const int cr = idx / (kD / 8), c = idx % (kD / 8);
+          const int rr = r0 + cr, node = rr / G, hh = rr % G;
+          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                (((size_t)b * a.Nmax + node) * a.Hq + g * G + hh) * kD;
+          reinterpret_cast<uint4*>(orow)[c] = *reinterpret_cast<const uint4*>(sStage + (size_t)cr * kStageH + c * 16);
+        }
+      } else {
+        float* wo = reinterpret_cast<float*>(a.workspace);
+        const size_t base = (((size_t)b * a.Hkv + g) * u.splits + split) * u.Rmax + r0;
+        for (int idx = tid; idx < nrows * (kD / 4); idx += kThreadsU) {
+          const int cr = idx / (kD / 4), c = idx % (kD / 4);
+          reinterpret_cast<float4*>(wo + (base + cr) * kD)[c] =
+              *reinterpret_cast<const float4*>(sStage + (size_t)cr * kStageF + c * 16);
+        }
       }
     }
   } else {
@@ -742,47 +769,14 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       tc_commit(&bars.fin);
       mbar_wait(&bars.fin, 0, u.wait);
     }
-    for (int i = tid; i < kRows; i += kThreadsU) s_mlc[i] = make_float2(-INFINITY, 0.f);
-    if (direct) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
-  }
-  if (!direct) {
-    // ------------------------------------------------------------ cluster merge of the split partials
-    // Each CTA of the cluster merges an equal share of the rows: for row r, with partials
-    // (O_s, M_s, l_s) of the cluster's CTAs s, out = sum_s 2^(M_s - M) O_s / sum_s 2^(M_s - M) l_s,
-    // M = max_s M_s, read from the peers' shared memory (distributed shared memory).  Two cluster
-    // barriers: partials complete before any read, reads complete before any CTA leaves.  Every CTA
-    // reaches both (all waits above are bounded).
-    cg::cluster_group cl = cg::this_cluster();
-    if (tid == 0) s_bad = (s_abort || s_err || entry_flag) ? 1 : 0;
-    __syncthreads();
-    cl.sync();
-    int anybad = 0;
-    for (int s2 = 0; s2 < u.csize; ++s2) anybad |= *cl.map_shared_rank(&s_bad, s2);
-    const int nrows = r_hi - r0;
-    const int q_lo = (int)((long long)split * nrows / u.csize);
-    const int q_hi = (int)((long long)(split + 1) * nrows / u.csize);
-    for (int crow = q_lo + warp; crow < q_hi; crow += kThreadsU / 32) {
-      float2 ml = make_float2(-INFINITY, 0.f);
-      if (lane < u.csize) ml = *cl.map_shared_rank(&s_mlc[crow], lane);
-      const float M = warp_max(ml.x);
-      const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-      const float L = warp_sum(ml.y * w);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s2 = 0; s2 < u.csize; ++s2) {
-        const float ws = __shfl_sync(0xffffffffu, w, s2);
-        if (ws == 0.f) continue;   // an empty or unusable partial (its rows may hold anything)
-        const float4 x = cl.map_shared_rank(reinterpret_cast<const float4*>(sStage + (size_t)crow * kStageF), s2)[lane];
-        acc.x = fmaf(x.x, ws, acc.x), acc.y = fmaf(x.y, ws, acc.y);
-        acc.z = fmaf(x.z, ws, acc.z), acc.w = fmaf(x.w, ws, acc.w);
-      }
-      const float inv = (L > 0.f && !anybad) ? 1.f / L : 0.f;
-      const int rr = r0 + crow, node = rr / G, hh = rr % G;
-      const size_t orow = (((size_t)b * a.Nmax + node) * a.Hq + g * G + hh);
-      reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + orow * kD)[lane] =
-          make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-      if (a.lse && lane == 0) a.lse[orow] = (L > 0.f && !anybad) ? (M + __log2f(L)) * kLn2 : 0.f;
+    if (direct) {
+      zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
+    } else {   // an unusable partial: the merge skips it (and zeroes the rows: status is flagged)
+      float* wml = reinterpret_cast<float*>(a.workspace) + (size_t)a.B * a.Hkv * u.splits * u.Rmax * kD;
+      const size_t base = (((size_t)b * a.Hkv + g) * u.splits + split) * u.Rmax;
+      for (int r = r0 + tid; r < r_hi; r += kThreadsU)
+        *reinterpret_cast<float2*>(wml + (base + r) * 2) = make_float2(-INFINITY, 0.f);
     }
-    cl.sync();
   }
   tc_fence_before();
   __syncthreads();
@@ -832,55 +826,13 @@ bool umma_eligible(const AttnArgs& a, tsd_dtype dtype) {
   return encoder() != nullptr;
 }
 
-// Largest cluster size <= want (halving) whose clusters the device can hold at least one of with
-// this kernel and shared-memory size; sizes above 8 need the non-portable opt-in.  Answers are
-// cached per (kernel, size, shared memory).
-int cluster_fit(const void* kernel, int want, size_t smem, int mtiles, int Hkv, int B) {
-  static std::mutex mu;
-  struct Key {
-    const void* k;
-    int c;
-    size_t s;
-    bool ok;
-  };
-  static Key memo[64];
-  static int nmemo = 0;
-  while (want > 1) {
-    bool ok = false, found = false;
-    {
-      std::lock_guard<std::mutex> lock(mu);
-      for (int i = 0; i < nmemo; ++i)
-        if (memo[i].k == kernel && memo[i].c == want && memo[i].s == smem) ok = memo[i].ok, found = true;
-    }
-    if (!found) {
-      if (want > 8) cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(mtiles * want, Hkv, B);
-      cfg.blockDim = dim3(kThreadsU);
-      cfg.dynamicSmemBytes = smem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = want, attr[0].val.clusterDim.y = 1, attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      ok = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n >= 1;
-      cudaGetLastError();
-      std::lock_guard<std::mutex> lock(mu);
-      if (nmemo < 64) memo[nmemo++] = Key{kernel, want, smem, ok};
-    }
-    if (ok) return want;
-    want = want > 8 ? 8 : want / 2;
-  }
-  return 1;
-}
-
 tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   UParams u{};
-  u.csize = p.csize, u.mtiles = p.umtiles;
+  u.splits = p.splits, u.Rmax = p.Rmax, u.mtiles = p.umtiles;
   u.wait = kWaitCycles;
   u.withhold = -1;
+  u.lpt = a.B > 1 && a.B <= kThreadsU ? 1 : 0;
   // Test hook for the bounded waits: TSD_TEST_WITHHOLD_TILE=t makes the K producer of every CTA
   // skip key tile t (and every later one), so the waits on it give up after 10^5 cycles and the
   // call reports TSD_ERR_TIMEOUT in status[] instead of stalling.
@@ -941,21 +893,9 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   }
   auto kernel = p.dual ? attn_umma_kernel<true> : attn_umma_kernel<false>;
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (!u.stage) u.csize = 1;   // the cluster merge stages partial rows in the idle K/V rings
-  u.csize = cluster_fit(reinterpret_cast<const void*>(kernel), u.csize, smem, u.mtiles, a.Hkv, a.B);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(u.mtiles * u.csize, a.Hkv, a.B);
-  cfg.blockDim = dim3(kThreadsU);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = u.csize, attr[1].val.clusterDim.y = 1, attr[1].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = u.csize > 1 ? 2 : 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, mkt, mvt, a, u) != cudaSuccess) return TSD_ERR_CUDA;
+  dim3 grid(u.mtiles * u.splits, a.Hkv, a.B);
+  if (launch_pdl(kernel, grid, dim3(kThreadsU), smem, stream, mq, mk, mv, mkt, mvt, a, u) != cudaSuccess)
+    return TSD_ERR_CUDA;
   return TSD_OK;
 }
 

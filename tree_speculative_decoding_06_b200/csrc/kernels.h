@@ -50,7 +50,7 @@ struct AttnPlan {
   int tps = 1, splits = 1;  // tiles per split, splits per (sequence, KV head, row tile)
   bool dual = false;        // tcgen05 kernel: two 128-row query tiles per CTA
   int umtiles = 0;          // tcgen05 kernel: row blocks per (sequence, KV head)
-  int csize = 1;            // tcgen05 kernel: CTAs (one cluster) splitting the keys of a row block
+  int usplits = 1;          // tcgen05 kernel: CTAs splitting a row block's keys (equal shares)
   int threads = 128;
   size_t smem = 0;
   size_t ws_bytes = 0;
@@ -76,7 +76,7 @@ struct AttnArgs {
   int32_t* status;
 };
 
-AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype);
+AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype, bool paged);
 tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream);
 // tcgen05 path (attn_umma.cu): bf16, d = 128, tree K/V in their own buffer, G a power of two.
 bool umma_eligible(const AttnArgs& a, tsd_dtype dtype);

@@ -80,11 +80,7 @@ class VerifyStep:
             self.out_tokens = torch.zeros(B, K + 1, **i32)
         self.history = torch.zeros(B, history_cap, **i32) if history_cap > 0 and self.fused else None
         self.history_len = torch.zeros(B, **i32) if self.history is not None else None
-        # the tcgen05 attention (bf16, d = 128, a power-of-two group) merges its key splits inside a
-        # cluster; the other attention kernels merge them in a second launch when the plan splits
-        G = Hq // Hkv
-        umma = dtype == torch.bfloat16 and d == 128 and G <= 128 and (G & (G - 1)) == 0
-        self.splits_merge = ws > 0 and not umma
+        self.splits_merge = ws > 0   # the plan splits the keys: a merge launch follows the attention
         if schedule == "overlap":
             self.side = torch.cuda.Stream(device=dev)
             self.ev_fork, self.ev_join = torch.cuda.Event(), torch.cuda.Event()
@@ -95,7 +91,7 @@ class VerifyStep:
         n = 2 + int(self.splits_merge)
         if self.accept == "greedy":
             return n + (2 if self.fused else 3)
-        return n + (3 if self.T > 0 else 2) + 1
+        return n + (4 if self.T > 0 else 2) + 1
 
     def attn_launches(self) -> int:
         """Kernels one attention call launches (the split kernel, and its merge when split)."""
