@@ -337,36 +337,51 @@ def measure(name, args, rank, world, dev, gpu_id):
     step_ms, attn_ms = reduce_over_ranks([step_ms, attn_ms], world, dev)
     bad = sum(int((st.status != 0).sum()) for st in steps)   # every sequence of every set must be clean
 
-    # end to end through the public API with host buffers: H2D of the step's inputs from pinned
-    # memory, the step, D2H of the accepted lengths / tokens / path
+    # end to end through the public API with host buffers: every step copies its inputs from pinned
+    # host memory (H2D), runs, and reads back the accepted lengths / tokens / path (D2H).  Two
+    # input buffers (the inputs only; the cache and prefix lengths are shared) and a copy stream
+    # let step i+1's H2D run while step i computes, as a serving loop would.
+    from tree_speculative_decoding_06_b200.step import VerifyStep as _VS
     keys_in = [k for k in ("q", "k_tree", "v_tree", "parent", "num_nodes", "tokens", "logits", "root_key", "z_p",
                            "z_q", "x", "u") if isinstance(x0.get(k), torch.Tensor)]
     host = {k: x0[k].cpu().pin_memory() for k in keys_in}
+    bufs = [sets[0], {**sets[0], **{k: sets[0][k].clone() for k in keys_in}}]
+    vsteps = [steps[0], _VS.for_inputs(bufs[1], dev)]
     outs = ["accept_len", "out_tokens"] + (["path"] if steps[0].path is not None else [])
-    host_out = {k: getattr(steps[0], k).cpu().pin_memory() for k in outs}
+    host_outs = [{k: getattr(vs, k).cpu().pin_memory() for k in outs} for vs in vsteps]
     h2d = sum(host[k].numel() * host[k].element_size() for k in keys_in)
-    d2h = sum(host_out[k].numel() * host_out[k].element_size() for k in outs)
+    d2h = sum(host_outs[0][k].numel() * host_outs[0][k].element_size() for k in outs)
     e_steps = max(10, min(args.steps, 200))
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
 
-    def e2e_step():
-        for k in keys_in:
-            sets[0][k].copy_(host[k], non_blocking=True)
-        one_step(0)
-        for k in outs:
-            host_out[k].copy_(getattr(steps[0], k), non_blocking=True)
+    def e2e_step(i):
+        j = i % 2
+        copy_stream.wait_event(done[j])          # step i-2 has finished with buffer j
+        with torch.cuda.stream(copy_stream):
+            for k in keys_in:
+                bufs[j][k].copy_(host[k], non_blocking=True)
+            copied[j].record(copy_stream)
+        stream.wait_event(copied[j])
+        with torch.cuda.stream(stream):
+            bufs[j]["prefix_len"].copy_(pl0[0], non_blocking=True)
+            vsteps[j].run(bufs[j])
+            for k in outs:
+                host_outs[j][k].copy_(getattr(vsteps[j], k), non_blocking=True)
+            done[j].record(stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            e2e_step()
+    for i in range(4):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e_steps):
-            e2e_step()
-        e1.record(stream)
+    e0.record(stream)
+    copy_stream.wait_event(e0)
+    for i in range(e_steps):
+        e2e_step(i)
+    e1.record(stream)
     torch.cuda.synchronize(dev)
     e_ms = reduce_over_ranks([e0.elapsed_time(e1) / e_steps], world, dev)[0]
 
@@ -387,16 +402,107 @@ def measure(name, args, rank, world, dev, gpu_id):
                    "parallelism": f"replicas over sequences x{world}"},
         "roofline": _roofline(inp, attn_ms, name) if rank == 0 else None,
         "e2e": {"value": round(aggregate_rate(tok, world, 1, e_ms), 1), "unit": "tokens/s",
+                "copies": "every step: H2D of its inputs from pinned memory, D2H of its results; the next "
+                          "step's H2D overlaps this step's compute (two input buffers)",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
         "status_errors": bad,
         "wall_s_timed": round(wall, 3),
     }
-    del g_steps, g_attn, sets, steps, x0, host, host_out
+    del g_steps, g_attn, sets, steps, x0, host, host_outs, bufs, vsteps
     torch.cuda.synchronize(dev)
     torch.cuda.empty_cache()
     return fields, inp
+
+
+def measure_extras(args, dev):
+    """The kernels beyond the verify step, each at its natural shape, timed as one CUDA graph of K
+    calls (CUDA events on the launching stream; inputs seeded, drawn on the device): the EAGLE-2
+    draft-tree expansion (B=16, F=K=10), stochastic multi-branch and threshold acceptance over the
+    eagle60 trees (B=16, N=60), and the SSD outcome-cache build (B=8, K=7 drafts, S=8 slots); all
+    over V=128256 bf16 logits.  Each reports microseconds per call and its algorithmic bytes
+    (the logits rows the call must read) as a fraction of the copy bandwidth."""
+    import torch
+
+    import tree_speculative_decoding_06_b200 as tsd
+    peak, peak_kind = read_peaks()
+    V = 128256
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+
+    def randn(*shape, sigma=1.0):
+        return (torch.randn(*shape, generator=gen, device=dev) * sigma).to(torch.bfloat16)
+
+    stream = torch.cuda.Stream(dev)
+
+    def timed(fn, n):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(n):
+                fn()
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+
+    def entry(ms, nbytes, what):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"us_per_call": round(ms * 1e3, 3), "algorithmic_bytes": int(nbytes), "achieved_gbs": round(gbs, 1),
+                "hbm_frac": round(gbs / peak, 4), "peak_kind": f"{peak_kind} hbm_gbs", "shape": what}
+
+    n = max(args.steps, 10)
+    out = {}
+    # draft tree expansion: capacity for every expansion the timing runs, so none overflows
+    B, F, K = 16, 10, 10
+    dt = tsd.DraftTree(B, F, 1 + (n + 4) * F * K, device=dev)
+    dlog = randn(B, F, V, sigma=3.0)
+    dt.init(torch.randint(0, V, (B,), device=dev, dtype=torch.int32, generator=gen))
+    ms = timed(lambda: dt.expand(dlog, K, stream=stream), n)
+    out["draft_tree_expand"] = entry(ms, B * F * V * 2, "B=16 F=10 K=10 V=128256 bf16")
+    # stochastic and threshold acceptance over the eagle60 trees
+    w = W.WORKLOADS["eagle60"].scaled(L=16, L_lo=8, V=256)
+    base = W.make_inputs(w, nan_guard=False)
+    N = base["parent"].shape[1]
+    parent = torch.from_numpy(base["parent"]).to(dev)
+    nn = torch.from_numpy(base["num_nodes"]).to(dev)
+    prep = tsd.tree_prepare(parent, nn, int(base["Dmax"]), False)
+    zp, zq = randn(w.B, N, V, sigma=2.0), None
+    zq = (zp.float() + torch.randn(w.B, N, V, generator=gen, device=dev) * 0.8).to(torch.bfloat16)
+    toks = torch.randint(0, V, (w.B, N), device=dev, dtype=torch.int32, generator=gen)
+    u = torch.rand(w.B, N, device=dev, generator=gen)
+    res = {}
+
+    def sample():
+        res["s"] = tsd.tree_accept_sample(zp, zq, toks, prep["parent_s"], u, 1.0, num_nodes=nn, Dmax=int(base["Dmax"]),
+                                          status=prep["status"], stream=stream)
+    ms = timed(sample, n)
+    A = res["s"]["accept_len"].cpu().numpy()
+    out["tree_accept_sample"] = entry(ms, int((A + 1).sum()) * 2 * V * 2,
+                                      "eagle60 trees B=16 N=60 V=128256 bf16 T=1 (bytes: the two rows of every "
+                                      "visited node)")
+    ms = timed(lambda: tsd.tree_accept_threshold(zp, toks, prep["parent_s"], 0.01, 1.0, num_nodes=nn,
+                                                 Dmax=int(base["Dmax"]), status=prep["status"], stream=stream), n)
+    out["tree_accept_threshold"] = entry(ms, w.B * N * V * 2, "eagle60 trees B=16 N=60 V=128256 bf16 tau=0.01")
+    # SSD outcome cache
+    Bs, Ks, S = 8, 7, 8
+    sl = randn(Bs, Ks + 1, V, sigma=3.0)
+    alpha = torch.rand(Bs, device=dev, generator=gen) * 0.5 + 0.4
+    us = torch.rand(Bs, Ks, device=dev, generator=gen)
+    ms = timed(lambda: tsd.ssd_cache_build(sl, alpha, 0.5, us, S, 1.0, stream=stream), n)
+    out["ssd_cache_build"] = entry(ms, Bs * (Ks + 1) * V * 2, "B=8 K=7 S=8 V=128256 bf16")
+    torch.cuda.synchronize(dev)
+    return out
 
 
 def run_ours(args, rank, world, local_rank):
@@ -429,6 +535,7 @@ def run_ours(args, rank, world, local_rank):
             per[name]["workload"] = f["config"]["workload"]
             res["gpu_launches"] += f["gpu_launches"]
         res["per_workload"] = per
+        res["next_kernels"] = measure_extras(args, dev)
     return res, inp
 
 

@@ -829,7 +829,7 @@ bool umma_eligible(const AttnArgs& a, tsd_dtype dtype) {
 tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   UParams u{};
-  u.splits = p.splits, u.Rmax = p.Rmax, u.mtiles = p.umtiles;
+  u.splits = p.usplits, u.Rmax = p.Rmax, u.mtiles = p.umtiles;
   u.wait = kWaitCycles;
   u.withhold = -1;
   u.lpt = a.B > 1 && a.B <= kThreadsU ? 1 : 0;

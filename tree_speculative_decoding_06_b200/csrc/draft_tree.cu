@@ -41,24 +41,39 @@ __device__ __forceinline__ bool better_node(double sa, int ia, double sb, int ib
   return sa > sb || (sa == sb && ia < ib);
 }
 
-// Insert (x, v) into the sorted (best first) list (tv, ti) of length K <= kMaxK: the new entry
-// bubbles in, the last one falls out.  Static indices only (the list stays in registers).
-__device__ __forceinline__ void topk_insert(float (&tv)[kMaxK], int (&ti)[kMaxK], int K, float x, int v) {
-#pragma unroll
-  for (int k = 0; k < kMaxK; ++k) {
-    if (k < K && better(x, v, tv[k], ti[k])) {
-      const float t = tv[k];
-      const int u = ti[k];
-      tv[k] = x, ti[k] = v;
-      x = t, v = u;
-    }
+// Warp-cooperative top-K (K <= kMaxK <= 32): lane k < K holds the warp's k-th best (value, index)
+// so far (best first; ties -> lower index).  A candidate enters only if it beats the K-th best, so
+// after the first few hundred tokens almost every 32-token batch is dismissed by one ballot; an
+// entry is placed by one ballot (its rank) and one shuffle (the lanes below it move down).
+struct WarpTopK {
+  float v;
+  int i;
+};
+
+__device__ __forceinline__ void wtopk_insert(WarpTopK& me, int K, int lane, float x, int xi) {
+  const bool ahead = lane < K && better(me.v, me.i, x, xi);
+  const int pos = __popc(__ballot_sync(0xffffffffu, ahead));
+  const float up_v = __shfl_up_sync(0xffffffffu, me.v, 1);
+  const int up_i = __shfl_up_sync(0xffffffffu, me.i, 1);
+  if (lane < K) {
+    if (lane == pos) me.v = x, me.i = xi;
+    else if (lane > pos) me.v = up_v, me.i = up_i;
   }
 }
-__device__ __forceinline__ void topk_at(const float (&tv)[kMaxK], const int (&ti)[kMaxK], int k, float& x, int& v) {
-  x = -INFINITY, v = INT_MAX;
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j)
-    if (j == k) x = tv[j], v = ti[j];
+
+// Offer each lane's candidate (x, xi) to the warp list; `thr` (the K-th best) is kept current.
+__device__ __forceinline__ void wtopk_offer(WarpTopK& me, WarpTopK& thr, int K, int lane, float x, int xi) {
+  unsigned want = __ballot_sync(0xffffffffu, better(x, xi, thr.v, thr.i));
+  while (want) {
+    const int src = __ffs(want) - 1;
+    const float cx = __shfl_sync(0xffffffffu, x, src);
+    const int ci = __shfl_sync(0xffffffffu, xi, src);
+    wtopk_insert(me, K, lane, cx, ci);
+    thr.v = __shfl_sync(0xffffffffu, me.v, K - 1);
+    thr.i = __shfl_sync(0xffffffffu, me.i, K - 1);
+    want &= want - 1;
+    want &= __ballot_sync(0xffffffffu, better(x, xi, thr.v, thr.i));
+  }
 }
 
 template <typename T>
@@ -68,38 +83,41 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
   const int c = blockIdx.x, f = blockIdx.y, b = blockIdx.z;
   const T* row = logits + ((size_t)b * F + f) * V;
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
-  float tv[kMaxK];
-  int ti[kMaxK];
-#pragma unroll
-  for (int k = 0; k < kMaxK; ++k) tv[k] = -INFINITY, ti[k] = INT_MAX;
-  float thr_v = -INFINITY;   // the K-th best so far
-  int thr_i = INT_MAX;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  WarpTopK me{-INFINITY, INT_MAX}, thr{-INFINITY, INT_MAX};
   float m = -INFINITY;
-  auto take = [&](float x, int v) {
-    m = fmaxf(m, x);
-    if (better(x, v, thr_v, thr_i)) {
-      topk_insert(tv, ti, K, x, v);
-      topk_at(tv, ti, K - 1, thr_v, thr_i);
-    }
-  };
   if (vec) {
-    for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
+    for (int v0 = lo; v0 < hi; v0 += kThreads * 8) {   // every lane of a warp runs the same trips
+      const int v = v0 + threadIdx.x * 8;
       float x[8];
-      load8<T>(row, v, x);
+      if (v < hi) {
+        load8<T>(row, v, x);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) take(x[e], v + e);
+        for (int e = 0; e < 8; ++e) x[e] = -INFINITY;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        m = fmaxf(m, x[e]);
+        wtopk_offer(me, thr, K, lane, x[e], v < hi ? v + e : INT_MAX);
+      }
     }
   } else {
-    for (int v = lo + threadIdx.x; v < hi; v += kThreads) take(load1(row, v), v);
+    for (int v0 = lo; v0 < hi; v0 += kThreads) {
+      const int v = v0 + threadIdx.x;
+      const float x = v < hi ? load1(row, v) : -INFINITY;
+      m = fmaxf(m, x);
+      wtopk_offer(me, thr, K, lane, x, v < hi ? v : INT_MAX);
+    }
   }
   // chunk maximum
   __shared__ float s_m[kThreads / 32];
   __shared__ double s_s[kThreads / 32];
-  __shared__ float s_bv[kThreads / 32];
-  __shared__ int s_bi[kThreads / 32], s_bt[kThreads / 32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float s_wv[kThreads / 32][kMaxK];
+  __shared__ int s_wi[kThreads / 32][kMaxK];
   float wm = warp_max(m);
   if (lane == 0) s_m[warp] = wm;
+  if (lane < K) s_wv[warp][lane] = me.v, s_wi[warp][lane] = me.i;
   __syncthreads();
   float M = -INFINITY;
 #pragma unroll
@@ -111,8 +129,10 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
       for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
         float x[8];
         load8<T>(row, v, x);
+        float t = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sum += (double)expf(x[e] - M);
+        for (int e = 0; e < 8; ++e) t += expf(x[e] - M);
+        sum += (double)t;
       }
     } else {
       for (int v = lo + threadIdx.x; v < hi; v += kThreads) sum += (double)expf(load1(row, v) - M);
@@ -121,34 +141,16 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (lane == 0) s_s[warp] = sum;
-  // chunk top-K: K rounds of a block argmax over every thread's current head
+  // chunk top-K: warp 0 offers the other warps' lists to its own, K candidates per lane batch
   __shared__ float s_topv[kMaxK];
   __shared__ int s_topi[kMaxK];
-  int h = 0;
-  for (int r = 0; r < K; ++r) {
-    float hv;
-    int hi_;
-    if (h < K) topk_at(tv, ti, h, hv, hi_);
-    else hv = -INFINITY, hi_ = INT_MAX;
-    float bv = hv;
-    int bi = hi_, bt = threadIdx.x;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      const int ot = __shfl_xor_sync(0xffffffffu, bt, o);
-      if (better(ov, oi, bv, bi)) bv = ov, bi = oi, bt = ot;
+  if (warp == 0) {
+    for (int w = 1; w < kThreads / 32; ++w) {
+      const float x = lane < K ? s_wv[w][lane] : -INFINITY;
+      const int xi = lane < K ? s_wi[w][lane] : INT_MAX;
+      wtopk_offer(me, thr, K, lane, x, xi);
     }
-    __syncthreads();   // s_bv of the previous round has been read
-    if (lane == 0) s_bv[warp] = bv, s_bi[warp] = bi, s_bt[warp] = bt;
-    __syncthreads();
-    float gv = -INFINITY;
-    int gi = INT_MAX, gt = -1;
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w)
-      if (better(s_bv[w], s_bi[w], gv, gi)) gv = s_bv[w], gi = s_bi[w], gt = s_bt[w];
-    if (threadIdx.x == gt) ++h;
-    if (threadIdx.x == 0) s_topv[r] = gv, s_topi[r] = gi;
+    if (lane < K) s_topv[lane] = me.v, s_topi[lane] = me.i;
   }
   __syncthreads();
   pdl_wait();   // the previous expansion may still be reading the workspace
