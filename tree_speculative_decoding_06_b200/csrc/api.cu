@@ -99,7 +99,7 @@ tsd_status tsd_tree_verify_attn(const void* q, const void* k_cache, const void* 
   a.max_blocks = 0, a.block_shift = 0, a.num_blocks = 0, a.Lcap = Lmax, a.prefix_len = prefix_len;
   a.k_tree = k_tree, a.v_tree = v_tree, a.parent_s = parent_s, a.num_nodes = num_nodes;
   a.B = B, a.Nmax = Nmax, a.Hq = Hq, a.Hkv = Hkv, a.d = d, a.Dmax = Dmax, a.scale = scale;
-  a.out = out, a.lse = lse, a.workspace = workspace, a.status = status;
+  a.out = out, a.lse = lse, a.workspace = workspace, a.ws_bytes = ws_bytes, a.status = status;
   return launch_attention(a, dtype, S(stream));
 }
 
@@ -127,7 +127,7 @@ tsd_status tsd_tree_verify_attn_paged(const void* q, const void* k_pages, const 
   a.Lcap = max_blocks * block_size, a.prefix_len = prefix_len;
   a.k_tree = k_tree, a.v_tree = v_tree, a.parent_s = parent_s, a.num_nodes = num_nodes;
   a.B = B, a.Nmax = Nmax, a.Hq = Hq, a.Hkv = Hkv, a.d = d, a.Dmax = Dmax, a.scale = scale;
-  a.out = out, a.lse = lse, a.workspace = workspace, a.status = status;
+  a.out = out, a.lse = lse, a.workspace = workspace, a.ws_bytes = ws_bytes, a.status = status;
   return launch_attention(a, dtype, S(stream));
 }
 

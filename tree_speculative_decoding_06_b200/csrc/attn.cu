@@ -620,7 +620,14 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
 
 tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream) {
   if (a.B == 0 || a.Nmax == 0) return TSD_OK;
-  const AttnPlan p = plan_attention(a.B, a.Nmax, a.Hq, a.Hkv, a.d, a.Lcap, dtype, a.block_table != nullptr);
+  AttnPlan p = plan_attention(a.B, a.Nmax, a.Hq, a.Hkv, a.d, a.Lcap, dtype, a.block_table != nullptr);
+  // TSD_ATTN_SPLITS=n overrides the tcgen05 kernel's split count (a tuning knob for sweeps), when
+  // the workspace the caller passed holds n partials
+  if (const char* e = getenv("TSD_ATTN_SPLITS")) {
+    const int n = atoi(e);
+    const size_t need = (size_t)a.B * a.Hkv * (size_t)n * p.Rmax * (a.d + 2) * sizeof(float);
+    if (n >= 1 && n <= 64 && (n == 1 || need <= a.ws_bytes)) p.usplits = n;
+  }
   dim3 grid(p.mtiles * p.splits, a.Hkv, a.B);
   // TSD_ATTN_PATH=mma selects the warp-level kernel even where the tcgen05 kernel applies (A/B runs)
   const char* path_env = getenv("TSD_ATTN_PATH");

@@ -204,7 +204,6 @@ __global__ void __launch_bounds__(kThreadsU, 1)
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
                      const __grid_constant__ CUtensorMap tmVt, const AttnArgs a, const UParams u) {
   pdl_trigger();
-  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ Bars bars;
@@ -216,6 +215,43 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   constexpr int kRows = kDual ? 2 * kBM : kBM;   // query rows of this CTA
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // ---------------------------------------------------------------- set-up
+  // Barriers, tensor memory and the tensor-map descriptors need nothing an earlier kernel writes,
+  // so they are set up before the wait on the previous launch (programmatic dependent launch):
+  // under a chain of kernels this prologue overlaps the previous kernel's tail.
+  if (tid == 0) {
+    mbar_init(&bars.q_full, kDual ? 8 : 1);   // two query tiles: each softmax warp stores its rows
+    for (int s = 0; s < u.ks; ++s) mbar_init(&bars.k_full[s], 1), mbar_init(&bars.k_empty[s], 1);
+    for (int s = 0; s < u.vs; ++s) mbar_init(&bars.v_full[s], 1), mbar_init(&bars.v_empty[s], 1);
+    for (int sb = 0; sb < kSBufs; ++sb) mbar_init(&bars.s_full[sb], 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bars.p_full[w], 4);
+      mbar_init(&bars.pv_done[w], 1);
+    }
+    mbar_init(&bars.mask_full, 1);
+    mbar_init(&bars.fin, 1);
+    s_err = 0;
+    s_abort = 0;
+    s_k_issued = s_v_issued = s_k_consumed = s_v_consumed = 0;
+    fence_barrier_init();
+    fence_proxy_async();
+    prefetch_tmap(&tmQ), prefetch_tmap(&tmK), prefetch_tmap(&tmV), prefetch_tmap(&tmKt), prefetch_tmap(&tmVt);
+  }
+  if (warp == 3) {
+    tmem_alloc(&s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  pdl_wait();
+  // every early return below frees the tensor memory first (nothing has used it yet)
+  auto leave = [&]() {
+    if (warp == 3) tmem_dealloc(tmem, kTmemCols);
+  };
+
   // CTA `split` of a (sequence, KV head, row block) takes an equal share of that sequence's own key
   // tiles (so ragged lengths stay balanced across its splits)
   const int split = blockIdx.x % u.splits, mt = blockIdx.x / u.splits;
@@ -241,7 +277,10 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   const int G = a.Hq / a.Hkv;
   const SeqView v = seq_view(a, b, G, kBN, 1 << 30);
   const int r0 = mt * kRows;
-  if (v.skip || r0 >= v.R) return;
+  if (v.skip || r0 >= v.R) {
+    leave();
+    return;
+  }
   const int r_hi = min(r0 + kRows, v.R);
   // a flagged or over-capacity sequence: zero rows (the split merge zeroes them too, as it reads
   // the status after every split has finished)
@@ -249,6 +288,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     if (split == 0) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
     if (split == 0 && mt == 0 && g == 0 && tid == 0 && a.status[b] == 0 && v.cap)
       flag_status(a.status, b, TSD_ERR_CAPACITY);
+    leave();
     return;
   }
   const bool direct = (u.splits == 1);
@@ -262,32 +302,6 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   uint8_t* sV = smem + u.v_off;
   uint32_t* sMask = reinterpret_cast<uint32_t*>(smem + u.mask_off);
 
-  // ---------------------------------------------------------------- set-up
-  if (tid == 0) {
-    mbar_init(&bars.q_full, kDual ? 8 : 1);   // two query tiles: each softmax warp stores its rows
-    for (int s = 0; s < u.ks; ++s) mbar_init(&bars.k_full[s], 1), mbar_init(&bars.k_empty[s], 1);
-    for (int s = 0; s < u.vs; ++s) mbar_init(&bars.v_full[s], 1), mbar_init(&bars.v_empty[s], 1);
-    for (int sb = 0; sb < kSBufs; ++sb) mbar_init(&bars.s_full[sb], 1);
-    for (int w = 0; w < 2; ++w) {
-      mbar_init(&bars.p_full[w], 4);
-      mbar_init(&bars.pv_done[w], 1);
-    }
-    mbar_init(&bars.mask_full, 1);
-    mbar_init(&bars.fin, 1);
-    s_err = 0;
-    s_abort = 0;
-    s_k_issued = s_v_issued = s_k_consumed = s_v_consumed = 0;
-    fence_barrier_init();
-    fence_proxy_async();
-  }
-  if (warp == 3) {
-    tmem_alloc(&s_tmem, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = s_tmem;
   float row_m = -INFINITY, row_l = 0.f;   // softmax threads: the row's final (max, sum) for their warpgroup
 
   if (warp == 0) {

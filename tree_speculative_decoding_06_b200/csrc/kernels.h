@@ -73,6 +73,7 @@ struct AttnArgs {
   void* out;
   float* lse;
   void* workspace;
+  size_t ws_bytes;
   int32_t* status;
 };
 
