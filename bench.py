@@ -624,6 +624,9 @@ def main():
                          "other workload under per_workload)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--next-only", action="store_true",
+                    help="measure only the kernels beyond the verify step (draft tree, tree sampling, threshold, "
+                         "SSD cache) and print them (profiling runs)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (small profiling captures only; the bench line "
                          "of a workload uses its own size)")
@@ -636,6 +639,11 @@ def main():
         res = run_reference(args, rank)
         if res is not None:
             print(json.dumps(res))
+        return
+    if args.next_only:
+        import torch
+        torch.cuda.set_device(local_rank)
+        print(json.dumps({"next_kernels": measure_extras(args, torch.device("cuda", local_rank))}))
         return
 
     import datetime

@@ -262,11 +262,14 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   int b = blockIdx.z;
   if (u.lpt) {
     __shared__ int s_b;
+    __shared__ int s_len[kThreadsU];
+    if (tid < a.B) s_len[tid] = a.prefix_len[tid];   // one read each, then ranks from shared memory
+    __syncthreads();
     if (tid < a.B) {
-      const int L = a.prefix_len[tid];
+      const int L = s_len[tid];
       int rank = 0;
       for (int o = 0; o < a.B; ++o) {
-        const int Lo = a.prefix_len[o];
+        const int Lo = s_len[o];
         rank += (Lo > L) || (Lo == L && o < tid);
       }
       if (rank == (int)blockIdx.z) s_b = tid;

@@ -211,9 +211,17 @@ __global__ void __launch_bounds__(kTS, 1) ssd_cache_kernel(const SSDArgs a) {
       for (int i = tid; i < 256; i += kTS) s_hist[i] = 0u;
       __syncthreads();
       const uint32_t hmask = shift + 8 >= 32 ? 0u : (0xffffffffu << (shift + 8));
-      for (int i = tid; i < cnt; i += kTS) {
-        const uint32_t k = okey(sZ[i]);
-        if ((k & hmask) == (prefix & hmask)) atomicAdd(&s_hist[(k >> shift) & 0xffu], 1u);
+      // warp-aggregated counting: logits crowd into a few high digits, so lanes with the same
+      // digit are grouped and their leader adds the group's size
+      for (int base = 0; base < cnt; base += kTS) {
+        const int i = base + tid;
+        int bin = -1;
+        if (i < cnt) {
+          const uint32_t k = okey(sZ[i]);
+          if ((k & hmask) == (prefix & hmask)) bin = (int)((k >> shift) & 0xffu);
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (uint32_t)__popc(peers));
       }
       __syncthreads();
       for (int i = tid; i < 256; i += kTS) s_xh[ph][i] = s_hist[i];

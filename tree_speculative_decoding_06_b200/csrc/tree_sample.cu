@@ -39,7 +39,7 @@ namespace {
 
 constexpr int kC = 8;           // CTAs per cluster (one sequence)
 constexpr int kTS = 512;        // threads per CTA
-constexpr int kMaxLevels = 256; // children tried at one node (a node with more flags the sequence)
+constexpr int kMaxChildren = 256; // children tried at one node (a node with more flags the sequence)
 constexpr double kLog2eD = 1.4426950408889634074;
 
 struct Temp {
@@ -123,15 +123,23 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
   return s;
 }
 
-// Target probability at level k of one token from its two logits: p_0 = softmax(zp / T), then
-// p_j = max(p_{j-1} - q, 0) / R_j.
-__device__ __forceinline__ double level_p(float zp, float zq, float Mp, double ip, float Mq, double iq, int k,
-                                          const double* R, const Temp& tc, double* q_out) {
-  double p = (double)expo(zp, Mp, tc) * ip;
-  const double q = k > 0 || q_out ? (double)expo(zq, Mq, tc) * iq : 0.0;
-  for (int j = 0; j < k; ++j) p = (p > q ? p - q : 0.0) / R[j];
+// The running target after k rejections at a node: p_0 = softmax(zp / T) and
+// p_j = max(p_{j-1} - q, 0) / R_j with R_j = sum_v max(p_{j-1} - q, 0).  By induction
+// p_k = max(p_0 - C_k q, 0) * D_k with C_0 = 0, D_0 = 1, C_{j+1} = C_j + 1 / D_j, D_{j+1} = D_j / R_{j+1}
+// (the same value as the step-by-step recursion up to rounding), so every level costs one
+// multiply-subtract per token instead of k divisions.
+struct Level {
+  double C, D;
+};
+
+__device__ __forceinline__ double level_p(float zp, float zq, float Mp, double ip, float Mq, double iq,
+                                          const Level& lv, const Temp& tc, double* q_out) {
+  const double p = (double)expo(zp, Mp, tc) * ip;
+  const bool need_q = lv.C != 0.0 || q_out;
+  const double q = need_q ? (double)expo(zq, Mq, tc) * iq : 0.0;
   if (q_out) *q_out = q;
-  return p;
+  const double r = p - lv.C * q;
+  return r > 0.0 ? r * lv.D : 0.0;
 }
 
 template <typename T>
@@ -151,7 +159,6 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
   __shared__ float s_redf[kTS / 32];
   __shared__ double s_redd[kTS / 32];
   __shared__ int s_wcnt[kTS / 32];
-  __shared__ double s_R[kMaxLevels];
   __shared__ int s_path[256];
   __shared__ int s_nchild, s_acc, s_tok;
   __shared__ double s_run[kTS];
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
       nc += tot;
       __syncthreads();
     }
-    if (nc > kMaxLevels) {   // more children than residual levels kept: the sequence is flagged
+    if (nc > kMaxChildren) {   // more children than the walk tries: the sequence is flagged
       too_wide = true;
       break;
     }
@@ -300,7 +307,8 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
     exchange_stats(mp, sp, mq, sq, Mp, Sp, Mq, Sq);
     const double ip = Sp > 0.0 ? 1.0 / Sp : 0.0, iq = Sq > 0.0 ? 1.0 / Sq : 0.0;
     // ---- children in order against the running residual
-    int k = 0, accepted = -1;
+    Level lv{0.0, 1.0};
+    int accepted = -1;
     const T* gp = reinterpret_cast<const T*>(a.zp) + ((size_t)b * a.Nmax + n) * V;
     const T* gq = reinterpret_cast<const T*>(a.zq) + ((size_t)b * a.Nmax + n) * V;
     for (int ci = 0; ci < nc; ++ci) {
@@ -310,7 +318,7 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
         bool acc = false;
         if (x >= 0 && x < V) {
           double qx;
-          const double px = level_p(ldf(gp + x), ldf(gq + x), Mp, ip, Mq, iq, k, s_R, a.tc, &qx);
+          const double px = level_p(ldf(gp + x), ldf(gq + x), Mp, ip, Mq, iq, lv, a.tc, &qx);
           acc = (double)ub[c] * qx < px;
         }
         s_acc = acc ? 1 : 0;
@@ -326,17 +334,13 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
       double r = 0.0;
       for (int i = tid; i < cnt; i += kTS) {
         double q;
-        const double p = level_p(ldf(sP + i), ldf(sQ + i), Mp, ip, Mq, iq, k, s_R, a.tc, &q);
+        const double p = level_p(ldf(sP + i), ldf(sQ + i), Mp, ip, Mq, iq, lv, a.tc, &q);
         r += p > q ? p - q : 0.0;
       }
       r = block_sum(r, s_redd);
       const double R = exchange_sum(r);
       __syncthreads();   // s_each is rewritten by the next exchange
-      if (R > 0.0) {
-        if (tid == 0) s_R[k] = R;
-        __syncthreads();
-        ++k;
-      }
+      if (R > 0.0) lv = Level{lv.C + 1.0 / lv.D, lv.D / R};
     }
     if (accepted >= 0) {
       ++depth;
@@ -352,7 +356,7 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
     double run = 0.0;
     int lastp = -1;
     for (int i = ra; i < re; ++i) {
-      const double p = level_p(ldf(sP + i), need_q ? ldf(sQ + i) : 0.f, Mp, ip, Mq, iq, k, s_R, a.tc, nullptr);
+      const double p = level_p(ldf(sP + i), need_q ? ldf(sQ + i) : 0.f, Mp, ip, Mq, iq, lv, a.tc, nullptr);
       if (p > 0.0) lastp = i;
       run += p;
     }
@@ -403,7 +407,7 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
         double c0 = s_run[tid];
         if (c0 <= t && ra < re && c0 + run > t) {
           for (int i = ra; i < re; ++i) {
-            c0 += level_p(ldf(sP + i), need_q ? ldf(sQ + i) : 0.f, Mp, ip, Mq, iq, k, s_R, a.tc, nullptr);
+            c0 += level_p(ldf(sP + i), need_q ? ldf(sQ + i) : 0.f, Mp, ip, Mq, iq, lv, a.tc, nullptr);
             if (c0 > t) {
               atomicMin(&s_tok, lo + i);
               break;
