@@ -86,20 +86,28 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpTopK me{-INFINITY, INT_MAX}, thr{-INFINITY, INT_MAX};
   float m = -INFINITY;
+  // 16-byte path: the thread's 64 logits of the chunk are loaded at once (one round trip to
+  // memory) and kept in registers for the maximum, the top-K offers and the exponential sum
+  constexpr int kGroups = kChunk / (kThreads * 8);
+  float xr[kGroups][8];
   if (vec) {
-    for (int v0 = lo; v0 < hi; v0 += kThreads * 8) {   // every lane of a warp runs the same trips
-      const int v = v0 + threadIdx.x * 8;
-      float x[8];
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int v = lo + (gi * kThreads + threadIdx.x) * 8;
       if (v < hi) {
-        load8<T>(row, v, x);
+        load8<T>(row, v, xr[gi]);
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = -INFINITY;
+        for (int e = 0; e < 8; ++e) xr[gi][e] = -INFINITY;
       }
+    }
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int v = lo + (gi * kThreads + threadIdx.x) * 8;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        m = fmaxf(m, x[e]);
-        wtopk_offer(me, thr, K, lane, x[e], v < hi ? v + e : INT_MAX);
+        m = fmaxf(m, xr[gi][e]);
+        wtopk_offer(me, thr, K, lane, xr[gi][e], v < hi ? v + e : INT_MAX);
       }
     }
   } else {
@@ -126,12 +134,11 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
   double sum = 0.0;
   if (M != -INFINITY) {
     if (vec) {
-      for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
-        float x[8];
-        load8<T>(row, v, x);
+#pragma unroll
+      for (int gi = 0; gi < kGroups; ++gi) {
         float t = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t += expf(x[e] - M);
+        for (int e = 0; e < 8; ++e) t += expf(xr[gi][e] - M);   // -inf padding adds 0
         sum += (double)t;
       }
     } else {

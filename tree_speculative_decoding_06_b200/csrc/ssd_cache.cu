@@ -104,7 +104,7 @@ __device__ void fanout(float alpha_in, int K, int S, int* n) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kTS, 1) ssd_cache_kernel(const SSDArgs a) {
+__global__ void __launch_bounds__(kTS, 2) ssd_cache_kernel(const SSDArgs a) {
   pdl_trigger();
   pdl_wait();
   cg::cluster_group cl = cg::this_cluster();
@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(kTS, 1) ssd_cache_kernel(const SSDArgs a) {
   __shared__ uint32_t s_hist[256];
   __shared__ uint32_t s_xh[2][256];      // histogram exchange slots
   __shared__ double s_xd[2];             // scalar exchange slots
+  __shared__ double2 s_xd2[2], s_xd2m;
   __shared__ float s_xf[2];
   __shared__ int s_xi[2];
   __shared__ uint32_t s_sel_key[kMaxS];  // this CTA's selected tokens
@@ -163,6 +164,22 @@ __global__ void __launch_bounds__(kTS, 1) ssd_cache_kernel(const SSDArgs a) {
     __syncthreads();
     ph ^= 1;
     return s;
+  };
+  auto sum_d2 = [&](double v0, double v1, double& t0, double& t1) {   // two cluster sums, one barrier
+    if (tid == 0) s_xd2[ph] = make_double2(v0, v1);
+    cl.sync();
+    if (tid == 0) {
+      double2 t = make_double2(0.0, 0.0);
+      for (int r = 0; r < kC; ++r) {
+        const double2 x = *cl.map_shared_rank(&s_xd2[ph], r);
+        t.x += x.x, t.y += x.y;
+      }
+      s_xd2m = t;
+    }
+    __syncthreads();
+    t0 = s_xd2m.x, t1 = s_xd2m.y;
+    __syncthreads();
+    ph ^= 1;
   };
   auto sum_i = [&](int v) -> int {         // cluster sum; s_eachi keeps the terms
     if (tid == 0) s_xi[ph] = v;
@@ -339,23 +356,26 @@ __global__ void __launch_bounds__(kTS, 1) ssd_cache_kernel(const SSDArgs a) {
   for (int i = 0; i < kTS / 32; ++i) mx = fmaxf(mx, s_redf[i]);
   __syncthreads();
   const float M = max_f(mx);
-  double se = 0.0;
-  for (int i = tid; i < cnt; i += kTS) se += (double)expo(ldf(sZ[i]), M, a.thi, a.tlo);
-  const double Sq = sum_d(block_sum(se));
-  const double iq = Sq > 0.0 ? 1.0 / Sq : 0.0;
   const double beta = a.beta;
   auto weight = [&](int i) -> double {
     const uint32_t k = okey(sZ[i]);
     return (na > 0 && (k > kth || (k == kth && i < tie_cut))) ? beta : 1.0;
   };
-  // s = sum of q w; q' = q w / s (q itself if s == 0)
-  double sw = 0.0;
-  for (int i = tid; i < cnt; i += kTS) sw += (double)expo(ldf(sZ[i]), M, a.thi, a.tlo) * iq * weight(i);
-  const double s = sum_d(block_sum(sw));
-  const bool plain = !(s > 0.0);
+  // With e = 2^((z - M) log2(e) / T): q = e / sum(e) and q' = q w / sum(q w) = e w / sum(e w), so
+  // both sums come from one pass (q itself when the weighted sum is 0).
+  double se = 0.0, sw = 0.0;
+  for (int i = tid; i < cnt; i += kTS) {
+    const double e = (double)expo(ldf(sZ[i]), M, a.thi, a.tlo);
+    se += e;
+    sw += e * weight(i);
+  }
+  double Sq, Sw;
+  sum_d2(block_sum(se), block_sum(sw), Sq, Sw);
+  const bool plain = !(Sw > 0.0);
+  const double inv = plain ? (Sq > 0.0 ? 1.0 / Sq : 0.0) : 1.0 / Sw;
   auto qprime = [&](int i) -> double {
-    const double q = (double)expo(ldf(sZ[i]), M, a.thi, a.tlo) * iq;
-    return plain ? q : q * weight(i) / s;
+    const double e = (double)expo(ldf(sZ[i]), M, a.thi, a.tlo);
+    return (plain ? e : e * weight(i)) * inv;
   };
   const int per = (cnt + kTS - 1) / kTS;
   const int ra = min(cnt, tid * per), re = min(cnt, ra + per);

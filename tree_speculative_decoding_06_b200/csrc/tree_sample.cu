@@ -123,6 +123,29 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
   return s;
 }
 
+// Block maxima / sums of two values at once (one pair of barriers for both).
+__device__ __forceinline__ void block_max2(float& a, float& b, float2* red) {
+  a = warp_max(a), b = warp_max(b);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = make_float2(a, b);
+  __syncthreads();
+  a = -INFINITY, b = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kTS / 32; ++i) a = fmaxf(a, red[i].x), b = fmaxf(b, red[i].y);
+}
+
+__device__ __forceinline__ void block_sum2(double& a, double& b, double2* red) {
+  a = warp_sum_d(a), b = warp_sum_d(b);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = make_double2(a, b);
+  __syncthreads();
+  a = 0.0, b = 0.0;
+#pragma unroll
+  for (int i = 0; i < kTS / 32; ++i) a += red[i].x, b += red[i].y;
+}
+
 // The running target after k rejections at a node: p_0 = softmax(zp / T) and
 // p_j = max(p_{j-1} - q, 0) / R_j with R_j = sum_v max(p_{j-1} - q, 0).  By induction
 // p_k = max(p_0 - C_k q, 0) * D_k with C_0 = 0, D_0 = 1, C_{j+1} = C_j + 1 / D_j, D_{j+1} = D_j / R_{j+1}
@@ -154,10 +177,14 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
   T* sP = reinterpret_cast<T*>(smem);
   T* sQ = sP + a.slice;
   int32_t* sChild = reinterpret_cast<int32_t*>(sQ + a.slice);   // a.Nmax entries
+  __shared__ float sCz[2 * kMaxChildren];                        // the children's (zp, zq) at their tokens
+  __shared__ uint8_t sCin[kMaxChildren];
   __shared__ Xch s_x[2];            // exchange slots, alternating (one barrier per exchange)
   __shared__ double s_xd[2];        // exchange slots of scalar sums (residual / slice mass)
   __shared__ float s_redf[kTS / 32];
   __shared__ double s_redd[kTS / 32];
+  __shared__ float2 s_redf2[kTS / 32];
+  __shared__ double2 s_redd2[kTS / 32];
   __shared__ int s_wcnt[kTS / 32];
   __shared__ int s_path[256];
   __shared__ int s_nchild, s_acc, s_tok;
@@ -293,15 +320,13 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
       mp = fmaxf(mp, ldf(sP + i));
       if (need_q) mq = fmaxf(mq, ldf(sQ + i));
     }
-    mp = block_max(mp, s_redf);
-    mq = block_max(mq, s_redf);
+    block_max2(mp, mq, s_redf2);
     double sp = 0.0, sq = 0.0;
     for (int i = tid; i < cnt; i += kTS) {
       if (mp != -INFINITY) sp += (double)expo(ldf(sP + i), mp, a.tc);
       if (need_q && mq != -INFINITY) sq += (double)expo(ldf(sQ + i), mq, a.tc);
     }
-    sp = block_sum(sp, s_redd);
-    sq = block_sum(sq, s_redd);
+    block_sum2(sp, sq, s_redd2);
     float Mp, Mq;
     double Sp, Sq;
     exchange_stats(mp, sp, mq, sq, Mp, Sp, Mq, Sq);
@@ -311,14 +336,23 @@ __global__ void __launch_bounds__(kTS, 1) tree_sample_kernel(const TSArgs a) {
     int accepted = -1;
     const T* gp = reinterpret_cast<const T*>(a.zp) + ((size_t)b * a.Nmax + n) * V;
     const T* gq = reinterpret_cast<const T*>(a.zq) + ((size_t)b * a.Nmax + n) * V;
+    // every child's token and two logits are gathered at once (one round trip), then tested in order
+    for (int ci = tid; ci < nc; ci += kTS) {
+      const int c = sChild[ci];
+      const int x = tok[c];
+      const bool in = x >= 0 && x < V;
+      sCz[2 * ci] = in ? ldf(gp + x) : 0.f;
+      sCz[2 * ci + 1] = in ? ldf(gq + x) : 0.f;
+      sCin[ci] = in ? 1 : 0;
+    }
+    __syncthreads();
     for (int ci = 0; ci < nc; ++ci) {
       const int c = sChild[ci];
       if (tid == 0) {
-        const int x = tok[c];
         bool acc = false;
-        if (x >= 0 && x < V) {
+        if (sCin[ci]) {
           double qx;
-          const double px = level_p(ldf(gp + x), ldf(gq + x), Mp, ip, Mq, iq, lv, a.tc, &qx);
+          const double px = level_p(sCz[2 * ci], sCz[2 * ci + 1], Mp, ip, Mq, iq, lv, a.tc, &qx);
           acc = (double)ub[c] * qx < px;
         }
         s_acc = acc ? 1 : 0;
