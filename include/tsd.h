@@ -21,7 +21,9 @@
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE memory owned by the caller; the library allocates
  *     nothing and keeps no state between calls.  Scratch ("workspace") is passed in; its size
- *     comes from the matching *_workspace_size() query, which is a pure host function.
+ *     comes from the matching *_workspace_size() query, which is a pure host function.  (The
+ *     attention's workspace is the one that carries something from call to call: ticket
+ *     words that every call returns to zero.)
  *   - Every call takes a CUDA stream (cudaStream_t passed as void*; NULL = legacy default
  *     stream), only enqueues work on it and returns without synchronising.  Accepted lengths
  *     and prefix lengths stay in device memory: nothing forces a device->host round trip
@@ -148,11 +150,23 @@ tsd_status tsd_tree_prepare(const int32_t *parent, const int32_t *num_nodes, int
  *   scale             score scale, usually 1/sqrt(d)
  *   out               [B, Nmax, Hq, d] dtype; rows of nodes i >= N_b are not written
  *   lse               [B, Nmax, Hq] fp32 or NULL: log-sum-exp of the scaled scores (natural log)
- *   workspace         device scratch of at least tsd_tree_verify_attn_workspace_size() bytes
- *                     (split-KV partials); may be NULL when that size is 0
+ *   workspace         device scratch of at least tsd_tree_verify_attn_workspace_size() bytes;
+ *                     may be NULL when that size is 0.  Its first
+ *                     tsd_tree_verify_attn_ticket_bytes() bytes are split-merge ticket words
+ *                     (the CTAs of one query block count themselves out and the last one
+ *                     merges the key splits): zero the workspace once (cudaMemset) before its
+ *                     first use; every call, error paths included, leaves them zero again.  A
+ *                     ticket word holding a count no call leaves flags TSD_ERR_WORKSPACE in
+ *                     status[b] and those rows are not written.  The rest holds the split-KV
+ *                     partials.  Calls in flight at the same time need separate workspaces.
+ *                     After a TSD_ERR_TIMEOUT, query blocks that had finished before the time-out
+ *                     may keep their rows: status[b] is what marks the sequence.
  *   status            [B] int32 (see the conventions above)
  * --------------------------------------------------------------------------------------- */
 size_t tsd_tree_verify_attn_workspace_size(int B, int Nmax, int Hq, int Hkv, int d, int Lmax, tsd_dtype dtype);
+
+/* Size of the ticket region at the start of an attention workspace (a constant). */
+size_t tsd_tree_verify_attn_ticket_bytes(void);
 
 tsd_status tsd_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache, int Lmax,
                                 const int32_t *prefix_len, const void *k_tree, const void *v_tree,

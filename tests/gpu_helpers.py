@@ -1,5 +1,7 @@
 """Shared helpers of the GPU parity tests: move generated inputs to the device, run the
 library through its binding, and compare with the oracle at the stated tolerances."""
+import os
+
 import numpy as np
 import torch
 
@@ -48,19 +50,40 @@ def gpu_prepare(x, forest):
     return tsd.tree_prepare(x["parent"], x["num_nodes"], int(x["Dmax"]), forest)
 
 
-def gpu_attention(inp, tree_in_cache=False, want_lse=True):
+def forced_split_workspace(inp):
+    """A zeroed workspace holding TSD_ATTN_SPLITS partials (the split-count knob only takes effect
+    when the workspace has room for them), or None when the knob is not set."""
+    n = int(os.environ.get("TSD_ATTN_SPLITS", "0"))
+    if n <= 1:
+        return None
+    B, Nmax, Hq, d = inp["q"].shape
+    Hkv = inp["k_tree"].shape[2]
+    dt = tsd.TSD_BF16 if dtype_of(inp) == "bf16" else tsd.TSD_F32
+    if "block_table" in inp:
+        planned = tsd.tree_verify_attn_paged_workspace_size(B, Nmax, Hq, Hkv, d, inp["block_table"].shape[1],
+                                                            inp["k_pages"].shape[2], dt)
+    else:
+        planned = tsd.tree_verify_attn_workspace_size(B, Nmax, Hq, Hkv, d, inp["k_cache"].shape[2], dt)
+    # at least what the planner asks for, or the binding would allocate a workspace of its own
+    nbytes = max(planned, tsd.tree_verify_attn_ticket_bytes() + B * Hkv * n * (Hq // Hkv) * Nmax * (d + 2) * 4)
+    return torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+
+
+def gpu_attention(inp, tree_in_cache=False, want_lse=True, workspace=None):
     x = to_device(inp)
     forest = bool(getattr(inp["workload"], "forest", False))
     prep = gpu_prepare(x, forest)
     kt, vt = (None, None) if tree_in_cache else (x["k_tree"], x["v_tree"])
+    if workspace is None:
+        workspace = forced_split_workspace(inp)
     if "k_pages" in x:
         out, lse = tsd.tree_verify_attn_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["prefix_len"],
                                               kt, vt, prep["parent_s"], x["num_nodes"], int(x["Dmax"]),
-                                              status=prep["status"], want_lse=want_lse)
+                                              status=prep["status"], want_lse=want_lse, workspace=workspace)
     else:
         out, lse = tsd.tree_verify_attn(x["q"], x["k_cache"], x["v_cache"], x["prefix_len"], kt, vt,
                                         prep["parent_s"], x["num_nodes"], int(x["Dmax"]), status=prep["status"],
-                                        want_lse=want_lse)
+                                        want_lse=want_lse, workspace=workspace)
     torch.cuda.synchronize()
     return to_np(out), (lse.cpu().numpy() if lse is not None else None), prep["status"].cpu().numpy()
 

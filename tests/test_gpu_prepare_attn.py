@@ -7,7 +7,7 @@ import torch
 import oracle
 import tree_speculative_decoding_06_b200 as tsd
 import workloads as W
-from gpu_helpers import check_attention, gpu_attention, lay_tree_in_cache, sample_rows
+from gpu_helpers import check_attention, forced_split_workspace, gpu_attention, lay_tree_in_cache, sample_rows
 from test_oracle_structure import all_trees
 
 pytestmark = pytest.mark.gpu
@@ -81,15 +81,35 @@ SMALL = {
 }
 
 
-@pytest.fixture(params=["auto", "mma"])
-def attn_path(request, monkeypatch):
-    """Run a test on the default kernel choice (tcgen05 where it applies) and again with the
-    warp-level mma.sync kernel forced, so both bf16 kernels stay covered."""
-    if request.param == "mma":
+def _use_path(monkeypatch, param):
+    for k in ("TSD_ATTN_PATH", "TSD_ATTN_SPLITS", "TSD_ATTN_MERGE"):
+        monkeypatch.delenv(k, raising=False)
+    if param == "mma":
         monkeypatch.setenv("TSD_ATTN_PATH", "mma")
-    else:
-        monkeypatch.delenv("TSD_ATTN_PATH", raising=False)
-    return request.param
+    if param.startswith("split3"):
+        monkeypatch.setenv("TSD_ATTN_SPLITS", "3")
+    if param.endswith("kernel"):
+        monkeypatch.setenv("TSD_ATTN_MERGE", "kernel")
+    elif param.startswith("split3") or param == "fused":
+        monkeypatch.setenv("TSD_ATTN_MERGE", "fused")
+    return param
+
+
+@pytest.fixture(params=["auto", "mma", "split3", "split3_merge_kernel"])
+def attn_path(request, monkeypatch):
+    """Run a test on the default kernel choice (tcgen05 where it applies), with the warp-level
+    mma.sync kernel forced, and with the tcgen05 kernel's keys split three ways, merged in the
+    kernel by the last CTA of each query block (forced for every shape) and by the separate merge
+    kernel, so every bf16 kernel and both merges stay covered."""
+    return _use_path(monkeypatch, request.param)
+
+
+@pytest.fixture(params=["auto", "mma", "merge_kernel", "fused"])
+def attn_path_full(request, monkeypatch):
+    """Full-size shapes at the planner's split counts (every bench shape splits its keys): the
+    default merge choice, the separate merge kernel and the in-kernel merge forced for every shape,
+    and the mma.sync kernel."""
+    return _use_path(monkeypatch, request.param)
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -165,7 +185,7 @@ FULL = ["tree26", "eagle60", "chain5", "forest"]
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_attention_full_size_sampled(name, attn_path):
+def test_attention_full_size_sampled(name, attn_path_full):
     w = W.WORKLOADS[name]
     inp = W.make_inputs(w)
     out, lse, st = gpu_attention(inp)
@@ -174,3 +194,31 @@ def test_attention_full_size_sampled(name, attn_path):
     check_attention(inp, out, lse, rows=rows)
     # properties at every row: finite, bounded by the largest |V| of the sequence's keys
     assert np.isfinite(out).all()
+
+
+def _ticket_words(ws):
+    return ws[:tsd.tree_verify_attn_ticket_bytes()].view(torch.int32)
+
+
+@pytest.mark.parametrize("name", ["tree26", "eagle60"])
+def test_merge_tickets_return_to_zero_and_garbage_is_reported(name, monkeypatch):
+    """The in-kernel split merge counts the CTAs of each query block on ticket words at the start of
+    the workspace: after a call they are all zero again, so back-to-back calls on one workspace
+    stay correct; a workspace whose ticket words were never zeroed is reported as
+    TSD_ERR_WORKSPACE in status[] (nothing is read or written out of place)."""
+    monkeypatch.setenv("TSD_ATTN_SPLITS", "3")
+    monkeypatch.setenv("TSD_ATTN_MERGE", "fused")
+    inp = W.make_inputs(SMALL[name])
+    ws = forced_split_workspace(inp)
+    for _ in range(3):
+        out, lse, st = gpu_attention(inp, workspace=ws)
+        assert (st == 0).all()
+        assert int(_ticket_words(ws).abs().sum()) == 0
+    check_attention(inp, out, lse)
+    ws[:tsd.tree_verify_attn_ticket_bytes()].fill_(0x7F)     # count 0x7f7f7f7f: no call leaves that
+    _, _, st = gpu_attention(inp, workspace=ws)
+    assert ((st & 0xFF) == 9).all(), st
+    ws.zero_()
+    out, lse, st = gpu_attention(inp, workspace=ws)
+    assert (st == 0).all()
+    check_attention(inp, out, lse)

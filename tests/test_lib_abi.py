@@ -66,7 +66,9 @@ def test_workspace_sizes_are_consistent():
     # contiguous one at the same capacity; both cover the partials of every split the plan makes
     a = tsd.tree_verify_attn_workspace_size(16, 60, 32, 8, 128, 8320, 1)
     b = tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1)
-    assert b >= a and b % (16 * 8 * 240 * 130 * 4) == 0
+    tk = tsd.tree_verify_attn_ticket_bytes()
+    assert tk >= 4 * 16 * 8 and tk % 256 == 0        # one ticket word per (sequence, KV head, row block)
+    assert b >= a and (b - tk) % (16 * 8 * 240 * 130 * 4) == 0
     assert tsd.tree_accept_greedy_workspace_size(8, 512, 128256) == 8 * 512 * 16 * 8
     assert tsd.chain_accept_sample_workspace_size(64, 5, 128256) > 64 * 11 * 16 * 8
 
@@ -104,8 +106,8 @@ def test_split_planner_choices_for_the_bench_workloads():
     fp32 per KV head and sequence) for the four bench shapes on a 148-SM device: tree26 9 (a sweep
     of 3..17 on B200 found 9 fastest), eagle60 3 (paged: planned for ragged lengths, each split an
     equal share of its own sequence, longest sequences first), chain5 2, forest 2."""
-    def splits(ws, B, Hkv, R, d=128):
-        return ws // (B * Hkv * R * (d + 2) * 4) if ws else 1
+    def splits(ws, B, Hkv, R, d=128):   # the ticket words come first, then the partials
+        return (ws - tsd.tree_verify_attn_ticket_bytes()) // (B * Hkv * R * (d + 2) * 4) if ws else 1
     assert splits(tsd.tree_verify_attn_workspace_size(1, 26, 32, 8, 128, 2112, 1), 1, 8, 104) == 9
     assert splits(tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1), 16, 8, 240) == 3
     assert splits(tsd.tree_verify_attn_workspace_size(64, 6, 64, 8, 128, 8256, 1), 64, 8, 48) == 2

@@ -39,6 +39,7 @@ _SIGS = {
     "tsd_tree_verify_attn": (_I, [_P, _P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
                                   _P, _SZ, _P, _P]),
     "tsd_tree_verify_attn_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "tsd_tree_verify_attn_ticket_bytes": (_SZ, []),
     "tsd_tree_verify_attn_paged": (_I, [_P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                         _I, _F, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_accept_greedy_workspace_size": (_SZ, [_I, _I, _I]),
@@ -165,11 +166,22 @@ def tree_verify_attn_paged_workspace_size(B, Nmax, Hq, Hkv, d, max_blocks, block
     return int(lib().tsd_tree_verify_attn_paged_workspace_size(B, Nmax, Hq, Hkv, d, max_blocks, block_size, dtype))
 
 
+def tree_verify_attn_ticket_bytes() -> int:
+    """Bytes of split-merge ticket words at the start of an attention workspace (kept zero)."""
+    return int(lib().tsd_tree_verify_attn_ticket_bytes())
+
+
+def _nbytes(ws) -> int:
+    """Bytes of a workspace tensor (0 for None): the size the C call is told it may use."""
+    return 0 if ws is None else ws.numel() * ws.element_size()
+
+
 def _ws(nbytes: int, like: torch.Tensor, ws):
+    # a new workspace starts zeroed: the attention's ticket words must be zero before first use
     if nbytes == 0:
         return ws
     if ws is None or ws.numel() * ws.element_size() < nbytes:
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=like.device)
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=like.device)
     return ws
 
 
@@ -192,7 +204,8 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent_s, 
     rc = lib().tsd_tree_verify_attn(_ptr(q), _ptr(k_cache), _ptr(v_cache), Lmax, _i32(prefix_len, "prefix_len"),
                                     _ptr(k_tree), _ptr(v_tree), _i32(parent_s, "parent_s"),
                                     _i32(num_nodes, "num_nodes"), B, Nmax, Hq, Hkv, d, Dmax, dt, float(scale),
-                                    _ptr(out), _ptr(lse), _ptr(workspace), nbytes, _ptr(status), _stream(stream))
+                                    _ptr(out), _ptr(lse), _ptr(workspace), _nbytes(workspace), _ptr(status),
+                                    _stream(stream))
     _check(rc, "tsd_tree_verify_attn")
     return out, lse
 
@@ -218,7 +231,7 @@ def tree_verify_attn_paged(q, k_pages, v_pages, block_table, prefix_len, k_tree,
                                           _i32(prefix_len, "prefix_len"), _ptr(k_tree), _ptr(v_tree),
                                           _i32(parent_s, "parent_s"), _i32(num_nodes, "num_nodes"), B, Nmax, Hq,
                                           Hkv, d, Dmax, dt, float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
-                                          nbytes, _ptr(status), _stream(stream))
+                                          _nbytes(workspace), _ptr(status), _stream(stream))
     _check(rc, "tsd_tree_verify_attn_paged")
     return out, lse
 

@@ -73,6 +73,8 @@ size_t tsd_tree_verify_attn_workspace_size(int B, int Nmax, int Hq, int Hkv, int
   return plan_attention(B, Nmax, Hq, Hkv, d, Lmax, dtype, false).ws_bytes;
 }
 
+size_t tsd_tree_verify_attn_ticket_bytes(void) { return kAttnTicketBytes; }
+
 size_t tsd_tree_verify_attn_paged_workspace_size(int B, int Nmax, int Hq, int Hkv, int d, int max_blocks,
                                                  int block_size, tsd_dtype dtype) {
   if (max_blocks < 0 || block_size <= 0) return 0;

@@ -614,27 +614,37 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
     }
   }
   const int wsplits = p.splits > p.usplits ? p.splits : p.usplits;   // either kernel may run
-  p.ws_bytes = wsplits > 1 ? (size_t)B * Hkv * wsplits * p.Rmax * (d + 2) * sizeof(float) : 0;
+  p.ws_bytes = wsplits > 1 ? kAttnTicketBytes + (size_t)B * Hkv * wsplits * p.Rmax * (d + 2) * sizeof(float) : 0;
   return p;
 }
 
-tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream) {
-  if (a.B == 0 || a.Nmax == 0) return TSD_OK;
-  AttnPlan p = plan_attention(a.B, a.Nmax, a.Hq, a.Hkv, a.d, a.Lcap, dtype, a.block_table != nullptr);
+tsd_status launch_attention(const AttnArgs& a_in, tsd_dtype dtype, cudaStream_t stream) {
+  if (a_in.B == 0 || a_in.Nmax == 0) return TSD_OK;
+  AttnPlan p = plan_attention(a_in.B, a_in.Nmax, a_in.Hq, a_in.Hkv, a_in.d, a_in.Lcap, dtype,
+                              a_in.block_table != nullptr);
   // TSD_ATTN_SPLITS=n overrides the tcgen05 kernel's split count (a tuning knob for sweeps), when
   // the workspace the caller passed holds n partials
   if (const char* e = getenv("TSD_ATTN_SPLITS")) {
     const int n = atoi(e);
-    const size_t need = (size_t)a.B * a.Hkv * (size_t)n * p.Rmax * (a.d + 2) * sizeof(float);
-    if (n >= 1 && n <= 64 && (n == 1 || need <= a.ws_bytes)) p.usplits = n;
+    const size_t need = kAttnTicketBytes + (size_t)a_in.B * a_in.Hkv * (size_t)n * p.Rmax * (a_in.d + 2) * sizeof(float);
+    if (n >= 1 && n <= 64 && (n == 1 || need <= a_in.ws_bytes)) p.usplits = n;
+  }
+  // the kernels see the partials; the ticket words stay at the start of the workspace
+  AttnArgs a = a_in;
+  int* tickets = nullptr;
+  if (a_in.workspace != nullptr && a_in.ws_bytes > kAttnTicketBytes) {
+    tickets = reinterpret_cast<int*>(a_in.workspace);
+    a.workspace = reinterpret_cast<uint8_t*>(a_in.workspace) + kAttnTicketBytes;
+    a.ws_bytes = a_in.ws_bytes - kAttnTicketBytes;
   }
   dim3 grid(p.mtiles * p.splits, a.Hkv, a.B);
   // TSD_ATTN_PATH=mma selects the warp-level kernel even where the tcgen05 kernel applies (A/B runs)
   const char* path_env = getenv("TSD_ATTN_PATH");
   const bool force_mma = path_env != nullptr && path_env[0] == 'm' && path_env[1] == 'm';
   if (dtype == TSD_BF16 && !force_mma && umma_eligible(a, dtype)) {
-    const tsd_status st = launch_attention_umma(a, p, stream);
-    if (st != TSD_OK || p.usplits <= 1) return st;
+    bool merged = false;
+    const tsd_status st = launch_attention_umma(a, p, tickets, &merged, stream);
+    if (st != TSD_OK || p.usplits <= 1 || merged) return st;
     const int rows_per_block = 8;
     dim3 cg((p.Rmax + rows_per_block - 1) / rows_per_block, a.Hkv, a.B);
     launch_pdl(attn_combine_kernel<128, __nv_bfloat16>, cg, dim3(256), 0, stream, a, p.BN, p.tps, p.usplits, p.Rmax,

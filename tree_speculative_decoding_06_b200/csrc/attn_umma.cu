@@ -83,6 +83,7 @@ struct UParams {
   int box_rows;        // rows per TMA box of the cache (64 contiguous, min(block, 64) paged)
   int W;               // ancestor-bit words per node
   int stage;           // epilogue rows go through shared memory (the ring region is large enough)
+  int* tickets;        // split merge in the kernel: one ticket word per row block (null: merge kernel)
   uint32_t k_off, v_off, mask_off, ps_off;   // shared-memory offsets
 };
 
@@ -198,6 +199,143 @@ __device__ __forceinline__ void load_tile(const AttnArgs& a, const SeqView& v, c
 // kDual: the CTA owns two 128-row query tiles of the same KV head and streams every K/V tile once
 // for both (warpgroup w owns query tile w over all key tiles); otherwise one query tile whose key
 // tiles alternate between the two warpgroups.
+// Split merge inside the kernel.  Every CTA of a (sequence, KV head, row block) publishes its
+// partial, then takes a ticket from the row block's word; the CTA that draws the last ticket merges
+// the partials and writes the output, and returns the word to zero for the next call.  No CTA
+// waits for another.  Returns 1 to the last CTA, 2 when the word held a count no call leaves
+// behind (the workspace was not zeroed before its first use), else 0.
+__device__ __forceinline__ int take_ticket(int* word, int splits, int* s_flag) {
+  __threadfence();   // this thread's partial stores, before the ticket
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int old = atomicAdd(word, 1);
+    const int r = old == splits - 1 ? 1 : ((old < 0 || old >= splits) ? 2 : 0);
+    if (r == 1) atomicExch(word, 0);
+    __threadfence();
+    *s_flag = r;
+  }
+  __syncthreads();
+  return *s_flag;
+}
+
+// The last CTA's merge (all threads).  (1) Every split's (max, sum) of every row into shared memory
+// with independent loads; (2) per row the largest split maximum, the splits' weights
+// 2^(M_s - M) / sum (s_w[s][row]) and the log-sum-exp; (3) every (row, 8 columns) the weighted sum
+// of the partial rows, four such pieces per thread and two splits per round so that many loads are
+// in flight, written as bf16.  This CTA's own partial is read from its staged rows in shared memory,
+// the others' from L2 (.cg: written by other SMs).  A split with no mass (M = -inf) has weight 0 and
+// its rows are never used.  Zero rows when the sequence is flagged or out of capacity.
+__device__ void merge_splits(const AttnArgs& a, const UParams& u, int b, int g, int G, int r0, int r_hi, int own,
+                             bool zero, const uint8_t* sStage, float* s_w, int rows_cap) {
+  if (zero) {
+    zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
+    return;
+  }
+  const int nrows = r_hi - r0, ns = u.splits, bd = blockDim.x;
+  const float* wo = reinterpret_cast<const float*>(a.workspace);
+  const float* wml = wo + (size_t)a.B * a.Hkv * ns * u.Rmax * kD;
+  const size_t base = ((size_t)b * a.Hkv + g) * ns * u.Rmax + r0;   // + s * Rmax + row
+  float2* s_ml = reinterpret_cast<float2*>(s_w + ns * rows_cap);      // [s][row]
+  const int npairs = ns * nrows;
+  for (int i0 = threadIdx.x; i0 < npairs; i0 += 4 * bd) {
+    float2 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int idx = i0 + j * bd, sp = idx / nrows, cr = idx - sp * nrows;
+      if (idx < npairs) v[j] = __ldcg(reinterpret_cast<const float2*>(wml + (base + (size_t)sp * u.Rmax + cr) * 2));
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int idx = i0 + j * bd, sp = idx / nrows, cr = idx - sp * nrows;
+      if (idx < npairs) s_ml[sp * rows_cap + cr] = v[j];
+    }
+  }
+  __syncthreads();
+  for (int cr = threadIdx.x; cr < nrows; cr += bd) {
+    float M = -INFINITY;
+    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, s_ml[sp * rows_cap + cr].x);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float l = 0.f;
+    for (int sp = 0; sp < ns; ++sp) {
+      const float2 ml = s_ml[sp * rows_cap + cr];
+      const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - Mu);
+      l += ml.y * w;
+      s_w[sp * rows_cap + cr] = w;
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    for (int sp = 0; sp < ns; ++sp) s_w[sp * rows_cap + cr] *= inv;
+    if (a.lse) {
+      const int r = r0 + cr;
+      a.lse[((size_t)b * a.Nmax + r / G) * a.Hq + g * G + r % G] = (M + __log2f(l)) * kLn2;
+    }
+  }
+  __syncthreads();
+  const int ntask = nrows * (kD / 8);
+  for (int t0 = threadIdx.x; t0 < ntask; t0 += 4 * bd) {
+    float acc[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + j * bd, cr = t / (kD / 8), c8 = t % (kD / 8);
+      const float w = t < ntask ? s_w[own * rows_cap + cr] : 0.f;
+      float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
+      if (t < ntask && w != 0.f) {
+        const float4* src = reinterpret_cast<const float4*>(sStage + (size_t)cr * kStageF + c8 * 32);
+        x0 = src[0], x1 = src[1];
+      }
+      acc[j][0] = w * x0.x, acc[j][1] = w * x0.y, acc[j][2] = w * x0.z, acc[j][3] = w * x0.w;
+      acc[j][4] = w * x1.x, acc[j][5] = w * x1.y, acc[j][6] = w * x1.z, acc[j][7] = w * x1.w;
+      if (w == 0.f)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+    }
+    for (int s0 = 0; s0 < ns; s0 += 2) {
+      float4 x[2][4][2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int sp = s0 + q;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = t0 + j * bd, cr = t / (kD / 8), c8 = t % (kD / 8);
+          if (sp < ns && sp != own && t < ntask) {
+            const float4* p4 = reinterpret_cast<const float4*>(wo + (base + (size_t)sp * u.Rmax + cr) * kD + c8 * 8);
+            x[q][j][0] = __ldcg(p4), x[q][j][1] = __ldcg(p4 + 1);
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int sp = s0 + q;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = t0 + j * bd, cr = t / (kD / 8);
+          if (sp < ns && sp != own && t < ntask) {
+            const float w = s_w[sp * rows_cap + cr];
+            if (w != 0.f) {
+              const float4 a0 = x[q][j][0], a1 = x[q][j][1];
+              acc[j][0] = fmaf(w, a0.x, acc[j][0]), acc[j][1] = fmaf(w, a0.y, acc[j][1]);
+              acc[j][2] = fmaf(w, a0.z, acc[j][2]), acc[j][3] = fmaf(w, a0.w, acc[j][3]);
+              acc[j][4] = fmaf(w, a1.x, acc[j][4]), acc[j][5] = fmaf(w, a1.y, acc[j][5]);
+              acc[j][6] = fmaf(w, a1.z, acc[j][6]), acc[j][7] = fmaf(w, a1.w, acc[j][7]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + j * bd, cr = t / (kD / 8), c8 = t % (kD / 8);
+      if (t < ntask) {
+        const int r = r0 + cr;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
+                              (((size_t)b * a.Nmax + r / G) * a.Hq + g * G + r % G) * kD;
+        *reinterpret_cast<uint4*>(orow + c8 * 8) =
+            make_uint4(pack_bf16x2(acc[j][0], acc[j][1]), pack_bf16x2(acc[j][2], acc[j][3]),
+                       pack_bf16x2(acc[j][4], acc[j][5]), pack_bf16x2(acc[j][6], acc[j][7]));
+      }
+    }
+  }
+}
+
 template <bool kDual>
 __global__ void __launch_bounds__(kThreadsU, 1)
     attn_umma_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -209,6 +347,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   __shared__ Bars bars;
   __shared__ uint32_t s_tmem;
   __shared__ int s_err;
+  __shared__ int s_ticket;
   __shared__ volatile int s_abort;
   __shared__ int s_k_issued, s_v_issued, s_k_consumed, s_v_consumed;
   __shared__ float2 s_ml1[kBM];   // warpgroup 1's (max, sum) per row, for the epilogue merge
@@ -278,7 +417,13 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     b = s_b;
   }
   const int G = a.Hq / a.Hkv;
-  const SeqView v = seq_view(a, b, G, kBN, 1 << 30);
+  SeqView v = seq_view(a, b, G, kBN, 1 << 30);
+  // the status word can be flagged by another CTA while this one starts: one read, shared by every
+  // thread, so the CTA takes one branch below
+  __shared__ int s_status;
+  if (tid == 0) s_status = __ldcg(a.status + b);
+  __syncthreads();
+  v.zero = v.cap || s_status != 0;
   const int r0 = mt * kRows;
   if (v.skip || r0 >= v.R) {
     leave();
@@ -287,10 +432,19 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   const int r_hi = min(r0 + kRows, v.R);
   // a flagged or over-capacity sequence: zero rows (the split merge zeroes them too, as it reads
   // the status after every split has finished)
+  // (the status word may be flagged while the launch runs, so with the merge in the kernel these
+  // CTAs still take their tickets: the row block's count must reach its split count)
   if (v.zero) {
-    if (split == 0) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
-    if (split == 0 && mt == 0 && g == 0 && tid == 0 && a.status[b] == 0 && v.cap)
+    if (split == 0 && mt == 0 && g == 0 && tid == 0 && s_status == 0 && v.cap)
       flag_status(a.status, b, TSD_ERR_CAPACITY);
+    if (u.splits > 1 && u.tickets != nullptr) {
+      int* word = u.tickets + ((size_t)b * a.Hkv + g) * u.mtiles + mt;
+      const int t = take_ticket(word, u.splits, &s_ticket);
+      if (t == 1) zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
+      else if (t == 2 && tid == 0) flag_status(a.status, b, TSD_ERR_WORKSPACE);
+    } else if (split == 0) {
+      zero_rows<__nv_bfloat16>(a, b, g, G, r0, r_hi);
+    }
     leave();
     return;
   }
@@ -795,6 +949,21 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         *reinterpret_cast<float2*>(wml + (base + r) * 2) = make_float2(-INFINITY, 0.f);
     }
   }
+  if (!direct && u.tickets != nullptr) {
+    int* word = u.tickets + ((size_t)b * a.Hkv + g) * u.mtiles + mt;
+    const int t = take_ticket(word, u.splits, &s_ticket);
+    if (t == 1) {
+      // one read of the status word for the whole CTA (another row block may flag it meanwhile);
+      // the staged rows hold this CTA's partial (none after a time-out: the status is flagged then)
+      __threadfence();
+      if (tid == 0) s_status = __ldcg(a.status + b);
+      __syncthreads();
+      merge_splits(a, u, b, g, G, r0, r_hi, split, s_abort != 0 || s_status != 0, sStage,
+                   reinterpret_cast<float*>(sStage + (size_t)kRows * kStageF), kRows);
+    } else if (t == 2 && tid == 0) {
+      flag_status(a.status, b, TSD_ERR_WORKSPACE);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 3) {
@@ -843,7 +1012,8 @@ bool umma_eligible(const AttnArgs& a, tsd_dtype dtype) {
   return encoder() != nullptr;
 }
 
-tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStream_t stream) {
+tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, int* tickets, bool* merged,
+                                 cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   UParams u{};
   u.splits = p.usplits, u.Rmax = p.Rmax, u.mtiles = p.umtiles;
@@ -876,6 +1046,20 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStrea
   u.mask_off = u.v_off + (uint32_t)u.vs * kSlot;
   u.ps_off = u.mask_off + ((mask_bytes + 15) & ~15u);
   u.stage = (uint32_t)(u.ks + u.vs) * kSlot >= (uint32_t)rows * kStageF ? 1 : 0;
+  // split merge in the kernel: the last CTA's staged rows and the splits' weights fit in the rings,
+  // and the ticket words fit their region.
+  // Measured on B200: it pays for the two-tile kernel (256 rows per CTA: the merge kernel re-reads
+  // large partials from DRAM after the grid ends), not for one-tile CTAs (many short CTAs pay the
+  // fence and ticket round trips; many splits leave one CTA a long merge), which keep the merge
+  // kernel.  TSD_ATTN_MERGE=kernel / =fused force either choice (A/B runs).
+  const char* merge_env = getenv("TSD_ATTN_MERGE");
+  const long long groups = (long long)a.B * a.Hkv * u.mtiles;
+  const bool want = merge_env != nullptr ? merge_env[0] == 'f' : p.dual;
+  const bool fuse = want && tickets != nullptr && u.splits > 1 && u.stage &&
+                    (size_t)(u.ks + u.vs) * kSlot >= (size_t)rows * kStageF + (size_t)u.splits * rows * 12 &&
+                    groups * 4 <= (long long)kAttnTicketBytes;
+  u.tickets = fuse ? tickets : nullptr;
+  *merged = fuse;
   const size_t smem = total(u.ks, u.vs);
 
   CUtensorMap mq, mk, mv, mkt, mvt;

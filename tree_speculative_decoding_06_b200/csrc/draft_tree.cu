@@ -26,6 +26,7 @@ constexpr int kThreads = 256;
 constexpr int kChunk = 16384;           // vocabulary entries per scan CTA
 constexpr int kMaxK = 16;               // children per node
 constexpr int kMaxFinalNodes = 4096;    // tree capacity finalize stages on chip
+constexpr int kMaxChunks = 64;          // vocabulary chunks per row (V <= 64 * kChunk)
 
 __host__ __device__ inline int dt_chunks(int V) { return (V + kChunk - 1) / kChunk; }
 // per (sequence, frontier row, chunk): fp64 sum, fp32 max, then K (value, index) pairs
@@ -76,6 +77,65 @@ __device__ __forceinline__ void wtopk_offer(WarpTopK& me, WarpTopK& thr, int K, 
   }
 }
 
+// One lane's share of the chunk's exponential sum, kept relative to a reference mt that is the same
+// for the whole warp (the warp's running maximum): st = sum of 2^((x - mt) log2(e)).  When the
+// warp's maximum grows, every lane rescales st by one fp64 exponential (a warp-uniform branch, a few
+// times per chunk), so the only fp32 rounding left is that of each token's own exponential.
+struct LaneSum {
+  float mt = -INFINITY;
+  double st = 0.0;
+};
+
+constexpr float kLog2eHi = 1.44269502162933349609375f;            // fp32 part of log2(e)
+constexpr float kLog2eLo = 1.925963033500011079198e-8f;           // log2(e) - kLog2eHi
+
+__device__ __forceinline__ float exp_rel(float x, float mt) {      // e^(x - mt), x <= mt
+  const float d = x - mt;
+  return exp2f(fmaf(d, kLog2eHi, d * kLog2eLo));
+}
+
+__device__ __forceinline__ void lane_sum_add8(LaneSum& ls, const float (&x)[8], float m8) {
+  const float wm8 = warp_max(m8);
+  if (wm8 > ls.mt) {
+    if (ls.st != 0.0) ls.st *= exp((double)ls.mt - (double)wm8);
+    ls.mt = wm8;
+  }
+  if (ls.mt == -INFINITY) return;
+  float t = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) t += exp_rel(x[e], ls.mt);            // -inf adds 0
+  ls.st += (double)t;
+}
+
+// Offer a group of 8 consecutive tokens (v .. v+7) per lane.  Each lane marks the tokens that reach
+// the warp's K-th best value; while any lane holds a mark, every such lane proposes its first one
+// and the proposals enter the list one at a time (exact comparison, lowest lane first), after which
+// the marks below the new K-th best are dropped.  Late in a chunk a group costs one compare per
+// token and one vote.
+__device__ __forceinline__ void offer8(WarpTopK& me, WarpTopK& thr, int K, int lane, const float (&x)[8], int v,
+                                       bool valid) {
+  unsigned cand = 0;
+  if (valid) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cand |= (x[e] >= thr.v ? 1u : 0u) << e;
+  }
+  while (__any_sync(0xffffffffu, cand != 0)) {
+    const int e = __ffs(cand) - 1;
+    float xv = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (e == j) xv = x[j];
+    const int xi = cand ? v + e : INT_MAX;
+    cand &= cand - 1;
+    wtopk_offer(me, thr, K, lane, xv, xi);
+    if (cand) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (x[j] < thr.v) cand &= ~(1u << j);
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict__ logits, int V, int F, int K,
                                                             int chunks, uint8_t* __restrict__ ws, int vec) {
@@ -85,86 +145,82 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpTopK me{-INFINITY, INT_MAX}, thr{-INFINITY, INT_MAX};
-  float m = -INFINITY;
-  // 16-byte path: the thread's 64 logits of the chunk are loaded at once (one round trip to
-  // memory) and kept in registers for the maximum, the top-K offers and the exponential sum
-  constexpr int kGroups = kChunk / (kThreads * 8);
-  float xr[kGroups][8];
+  LaneSum ls;
   if (vec) {
+    // 16-byte loads, the next group in flight while this one is scanned; every lane of a warp
+    // runs the same trips (a lane past the end offers nothing)
+    float x[8], y[8];
+    int v = lo + threadIdx.x * 8;
+    if (v < hi) load8<T>(row, v, x);
+#pragma unroll 1
+    for (; v - threadIdx.x * 8 < hi; v += kThreads * 8) {
+      const bool valid = v < hi;
+      const int vn = v + kThreads * 8;
+      if (vn < hi) load8<T>(row, vn, y);
+      if (!valid) {
 #pragma unroll
-    for (int gi = 0; gi < kGroups; ++gi) {
-      const int v = lo + (gi * kThreads + threadIdx.x) * 8;
-      if (v < hi) {
-        load8<T>(row, v, xr[gi]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xr[gi][e] = -INFINITY;
+        for (int e = 0; e < 8; ++e) x[e] = -INFINITY;
       }
-    }
+      float m8 = x[0];
 #pragma unroll
-    for (int gi = 0; gi < kGroups; ++gi) {
-      const int v = lo + (gi * kThreads + threadIdx.x) * 8;
+      for (int e = 1; e < 8; ++e) m8 = fmaxf(m8, x[e]);
+      offer8(me, thr, K, lane, x, v, valid);
+      lane_sum_add8(ls, x, m8);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        m = fmaxf(m, xr[gi][e]);
-        wtopk_offer(me, thr, K, lane, xr[gi][e], v < hi ? v + e : INT_MAX);
-      }
+      for (int e = 0; e < 8; ++e) x[e] = y[e];
     }
   } else {
     for (int v0 = lo; v0 < hi; v0 += kThreads) {
       const int v = v0 + threadIdx.x;
       const float x = v < hi ? load1(row, v) : -INFINITY;
-      m = fmaxf(m, x);
       wtopk_offer(me, thr, K, lane, x, v < hi ? v : INT_MAX);
+      const float wx = warp_max(x);
+      if (wx > ls.mt) {
+        if (ls.st != 0.0) ls.st *= exp((double)ls.mt - (double)wx);
+        ls.mt = wx;
+      }
+      if (ls.mt != -INFINITY) ls.st += (double)exp_rel(x, ls.mt);
     }
   }
-  // chunk maximum
+  // chunk maximum and sum: the warps' sums (relative to their maxima), then the block's maximum
   __shared__ float s_m[kThreads / 32];
   __shared__ double s_s[kThreads / 32];
   __shared__ float s_wv[kThreads / 32][kMaxK];
   __shared__ int s_wi[kThreads / 32][kMaxK];
-  float wm = warp_max(m);
-  if (lane == 0) s_m[warp] = wm;
+  const float wm = ls.mt;   // the same in every lane
+  double sum = ls.st;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) s_m[warp] = wm, s_s[warp] = sum;
   if (lane < K) s_wv[warp][lane] = me.v, s_wi[warp][lane] = me.i;
   __syncthreads();
   float M = -INFINITY;
 #pragma unroll
   for (int w = 0; w < kThreads / 32; ++w) M = fmaxf(M, s_m[w]);
-  // fp64 sum of fp32 exponentials relative to the chunk maximum (second pass, cache-resident)
-  double sum = 0.0;
-  if (M != -INFINITY) {
-    if (vec) {
-#pragma unroll
-      for (int gi = 0; gi < kGroups; ++gi) {
-        float t = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t += expf(xr[gi][e] - M);   // -inf padding adds 0
-        sum += (double)t;
-      }
-    } else {
-      for (int v = lo + threadIdx.x; v < hi; v += kThreads) sum += (double)expf(load1(row, v) - M);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) s_s[warp] = sum;
-  // chunk top-K: warp 0 offers the other warps' lists to its own, K candidates per lane batch
+  // chunk top-K: each of the 8 K warp candidates counts the candidates that beat it and, if fewer
+  // than K do, takes that slot (tokens are distinct across warps; unused slots keep (-inf, none))
   __shared__ float s_topv[kMaxK];
   __shared__ int s_topi[kMaxK];
-  if (warp == 0) {
-    for (int w = 1; w < kThreads / 32; ++w) {
-      const float x = lane < K ? s_wv[w][lane] : -INFINITY;
-      const int xi = lane < K ? s_wi[w][lane] : INT_MAX;
-      wtopk_offer(me, thr, K, lane, x, xi);
+  if (threadIdx.x < K) s_topv[threadIdx.x] = -INFINITY, s_topi[threadIdx.x] = INT_MAX;
+  __syncthreads();
+  if (threadIdx.x < (kThreads / 32) * K) {
+    const int w = threadIdx.x / K, j = threadIdx.x % K;
+    const float xv = s_wv[w][j];
+    const int xi = s_wi[w][j];
+    if (xi != INT_MAX) {
+      int rank = 0;
+      for (int w2 = 0; w2 < kThreads / 32; ++w2)
+        for (int j2 = 0; j2 < K; ++j2) rank += better(s_wv[w2][j2], s_wi[w2][j2], xv, xi) ? 1 : 0;
+      if (rank < K) s_topv[rank] = xv, s_topi[rank] = xi;
     }
-    if (lane < K) s_topv[lane] = me.v, s_topi[lane] = me.i;
   }
   __syncthreads();
   pdl_wait();   // the previous expansion may still be reading the workspace
   if (threadIdx.x == 0) {
     double S = 0.0;
 #pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) S += s_s[w];
+    for (int w = 0; w < kThreads / 32; ++w)
+      if (s_s[w] != 0.0) S += s_m[w] == M ? s_s[w] : s_s[w] * exp((double)s_m[w] - (double)M);
     uint8_t* rec = ws + (((size_t)b * F + f) * chunks + c) * dt_rec_bytes(K);
     ChunkRec cr;
     cr.s = S, cr.m = M, cr.pad = 0.f;
@@ -218,43 +274,60 @@ __global__ void __launch_bounds__(kThreads) draft_expand_kernel(DraftTreeArgs t,
     for (int i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = src[i];
   }
   __syncthreads();
-  // one thread per frontier row: merge the chunk records, append the row's K children
-  const int f = threadIdx.x;
-  if (f < nf) {
-    const uint8_t* recs = s_recs + (size_t)f * chunks * rb;
+  // the row maxima, then every (row, chunk) sum rescaled to its row's maximum in fp64, then per row
+  // the log-sum-exp (chunks summed in order)
+  __shared__ float s_M[kMaxK];
+  __shared__ double s_lse[kMaxK], s_psc[kMaxK];
+  __shared__ int s_par[kMaxK], s_pdep[kMaxK];
+  __shared__ double s_term[kMaxK * kMaxChunks];
+  auto rec_at = [&](int f, int c) { return s_recs + ((size_t)f * chunks + c) * rb; };
+  if (threadIdx.x < nf) {
+    const int f = threadIdx.x;
     float M = -INFINITY;
-    for (int c = 0; c < chunks; ++c) M = fmaxf(M, reinterpret_cast<const ChunkRec*>(recs + c * rb)->m);
-    double S = 0.0;
-    for (int c = 0; c < chunks; ++c) {
-      const ChunkRec* cr = reinterpret_cast<const ChunkRec*>(recs + c * rb);
-      if (cr->m != -INFINITY) S += cr->s * exp((double)cr->m - (double)M);
-    }
-    const double lse = (double)M + log(S);
+    for (int c = 0; c < chunks; ++c) M = fmaxf(M, reinterpret_cast<const ChunkRec*>(rec_at(f, c))->m);
+    s_M[f] = M;
     const int p = t.frontier[(size_t)b * t.F + f];
-    const double sp = t.score[base + p];
-    const int dp = t.depth[base + p];
-    int head[64];   // per-chunk read position of the K-way merge (chunks <= 64)
-    for (int c = 0; c < chunks; ++c) head[c] = 0;
-    for (int k = 0; k < K; ++k) {
-      float bv = -INFINITY;
-      int bi = INT_MAX, bc = -1;
-      for (int c = 0; c < chunks; ++c) {
-        if (head[c] >= K) continue;
-        const uint8_t* rec = recs + c * rb;
-        const float v = reinterpret_cast<const float*>(rec + 16)[head[c]];
-        const int i = reinterpret_cast<const int*>(rec + 16 + 4 * K)[head[c]];
-        if (i != INT_MAX && better(v, i, bv, bi)) bv = v, bi = i, bc = c;
-      }
-      if (bc >= 0) ++head[bc];
-      const int node = n0 + f * K + k;
-      const double sc = sp + ((double)bv - lse);
-      t.parent[base + node] = p;
-      t.token[base + node] = bi == INT_MAX ? 0 : bi;
-      t.score[base + node] = sc;
-      t.depth[base + node] = dp + 1;
-      s_sc[f * K + k] = sc;
-      s_id[f * K + k] = node;
+    s_par[f] = p, s_psc[f] = t.score[base + p], s_pdep[f] = t.depth[base + p];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < nf * chunks; idx += blockDim.x) {
+    const int f = idx / chunks, c = idx % chunks;
+    const ChunkRec* cr = reinterpret_cast<const ChunkRec*>(rec_at(f, c));
+    s_term[f * kMaxChunks + c] = cr->m != -INFINITY ? cr->s * exp((double)cr->m - (double)s_M[f]) : 0.0;
+  }
+  __syncthreads();
+  if (threadIdx.x < nf) {
+    const int f = threadIdx.x;
+    double S = 0.0;
+    for (int c = 0; c < chunks; ++c) S += s_term[f * kMaxChunks + c];
+    s_lse[f] = (double)s_M[f] + log(S);
+  }
+  __syncthreads();
+  // the row's K children: each chunk candidate counts the candidates of its row that beat it and,
+  // if fewer than K do, becomes that child (tokens are distinct across chunks, and the row holds
+  // at least K candidates since K <= V)
+  for (int idx = threadIdx.x; idx < nf * chunks * K; idx += blockDim.x) {
+    const int f = idx / (chunks * K), rem = idx % (chunks * K), c = rem / K, k = rem % K;
+    const uint8_t* rec = rec_at(f, c);
+    const float xv = reinterpret_cast<const float*>(rec + 16)[k];
+    const int xi = reinterpret_cast<const int*>(rec + 16 + 4 * K)[k];
+    if (xi == INT_MAX) continue;
+    int rank = 0;
+    for (int c2 = 0; c2 < chunks; ++c2) {
+      const uint8_t* r2 = rec_at(f, c2);
+      const float* v2 = reinterpret_cast<const float*>(r2 + 16);
+      const int* i2 = reinterpret_cast<const int*>(r2 + 16 + 4 * K);
+      for (int k2 = 0; k2 < K; ++k2) rank += (i2[k2] != INT_MAX && better(v2[k2], i2[k2], xv, xi)) ? 1 : 0;
     }
+    if (rank >= K) continue;
+    const int node = n0 + f * K + rank;
+    const double sc = s_psc[f] + ((double)xv - s_lse[f]);
+    t.parent[base + node] = s_par[f];
+    t.token[base + node] = xi;
+    t.score[base + node] = sc;
+    t.depth[base + node] = s_pdep[f] + 1;
+    s_sc[f * K + rank] = sc;
+    s_id[f * K + rank] = node;
   }
   __syncthreads();
   // new frontier: rank of every child among all children by (score desc, node index asc)

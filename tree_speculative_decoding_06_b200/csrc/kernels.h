@@ -38,6 +38,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The attention workspace starts with the split-merge ticket words (one int32 per (sequence, KV
+// head, row block) of the tcgen05 kernel, at most kAttnTicketBytes / 4 of them), zero between calls;
+// the partials follow.
+constexpr size_t kAttnTicketBytes = 65536;
+
 // Split-KV plan of one attention launch: a CTA covers BM query rows of one (sequence, KV head)
 // and `tps` key tiles of BN keys; the keys of sequence b are its prefix tiles followed by its
 // tree tiles.  Partials of (max, sum, unnormalised output) go to the workspace when a sequence
@@ -81,7 +86,10 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
 tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream);
 // tcgen05 path (attn_umma.cu): bf16, d = 128, tree K/V in their own buffer, G a power of two.
 bool umma_eligible(const AttnArgs& a, tsd_dtype dtype);
-tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, cudaStream_t stream);
+// `tickets` (may be null) enables the split merge inside the kernel; *merged says whether it ran
+// there (otherwise the caller launches the merge kernel).
+tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, int* tickets, bool* merged,
+                                 cudaStream_t stream);
 
 tsd_status launch_tree_prepare(const int32_t* parent, const int32_t* num_nodes, int B, int Nmax, int Dmax,
                                int forest, int32_t* parent_s, int32_t* depth, int32_t* anc, uint32_t* anc_bits,

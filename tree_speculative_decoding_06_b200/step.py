@@ -65,7 +65,7 @@ class VerifyStep:
             ws = tree_verify_attn_paged_workspace_size(B, Nmax, Hq, Hkv, d, max_blocks, block_size, dt)
         else:
             ws = tree_verify_attn_workspace_size(B, Nmax, Hq, Hkv, d, Lmax, dt)
-        self.attn_ws = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.zeros(max(ws, 1), dtype=torch.uint8, device=dev)   # ticket words start at zero
         if accept == "greedy":
             self.acc_ws = torch.empty(max(tree_accept_greedy_workspace_size(B, Nmax, V), 1), dtype=torch.uint8,
                                       device=dev)
