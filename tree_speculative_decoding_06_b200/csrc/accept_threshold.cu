@@ -42,8 +42,8 @@ __device__ __forceinline__ float expo(float z, float zm, float hi, float lo) {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) row_stats_chunks(const T* __restrict__ logits, int V, int rows_per_seq,
                                                              const int32_t* __restrict__ num_rows, int chunks,
-                                                             float thi, float tlo, RowStat* __restrict__ part,
-                                                             int vec) {
+                                                             float thi, float tlo, double cpow,
+                                                             RowStat* __restrict__ part, int vec) {
   pdl_trigger();
   const int c = blockIdx.x, i = blockIdx.y, b = blockIdx.z;
   const int n = num_rows ? num_rows[b] : rows_per_seq;
@@ -53,63 +53,75 @@ __global__ void __launch_bounds__(kThreads) row_stats_chunks(const T* __restrict
   }
   const T* row = logits + ((size_t)b * rows_per_seq + i) * V;
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float sv[kThreads / 32], sm[kThreads / 32];
+  __shared__ int si[kThreads / 32];
+  __shared__ double ss[kThreads / 32];
   float bv = -INFINITY;
   int bi = INT_MAX;
+  float wm;          // the warp's maximum: the reference of its exponential sum
+  double sum = 0.0;  // the warp's sum relative to wm (lane shares)
   if (vec) {
-    for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
-      float x[8];
-      load8<T>(row, v, x);
+    // 16-byte path: the thread's 32 logits of the chunk are loaded at once and stay in registers,
+    // so the sum is taken relative to the warp's maximum in the same pass
+    constexpr int kGroups = kChunk / (kThreads * 8);
+    float x[kGroups][8];
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int v = lo + (gi * kThreads + threadIdx.x) * 8;
+      if (v < hi) {
+        load8<T>(row, v, x[gi]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[gi][e] = -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int v = lo + (gi * kThreads + threadIdx.x) * 8;
 #pragma unroll
       for (int e = 0; e < 8; ++e)
-        if (x[e] > bv) bv = x[e], bi = v + e;
+        if (x[gi][e] > bv) bv = x[gi][e], bi = v + e;   // ascending order: ties keep the lower index
+    }
+    wm = warp_max(bv);
+    if (wm != -INFINITY) {
+#pragma unroll
+      for (int gi = 0; gi < kGroups; ++gi) {
+        float t = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t += expo(x[gi][e], wm, thi, tlo);   // -inf adds 0
+        sum += (double)t;
+      }
     }
   } else {
     for (int v = lo + threadIdx.x; v < hi; v += kThreads) {
       const float x = load1(row, v);
       if (better(x, v, bv, bi)) bv = x, bi = v;
     }
+    wm = warp_max(bv);
+    if (wm != -INFINITY)
+      for (int v = lo + threadIdx.x; v < hi; v += kThreads) sum += (double)expo(load1(row, v), wm, thi, tlo);
   }
-  // block argmax (ties -> lower index)
-  __shared__ float sv[kThreads / 32];
-  __shared__ int si[kThreads / 32];
-  __shared__ double ss[kThreads / 32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // block argmax (ties -> lower index) and maximum; the warps' sums rescaled to it in fp64
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
     const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
     if (better(ov, oi, bv, bi)) bv = ov, bi = oi;
   }
-  if (lane == 0) sv[warp] = bv, si[warp] = bi;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) sv[warp] = bv, si[warp] = bi, sm[warp] = wm, ss[warp] = sum;
   __syncthreads();
   float M = -INFINITY;
   int Mi = INT_MAX;
   for (int w = 0; w < kThreads / 32; ++w)
     if (better(sv[w], si[w], M, Mi)) M = sv[w], Mi = si[w];
-  // fp64 sum of the chunk's exponentials relative to M (second pass, cache-resident)
-  double sum = 0.0;
-  if (M != -INFINITY) {
-    if (vec) {
-      for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
-        float x[8];
-        load8<T>(row, v, x);
-        float t = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t += expo(x[e], M, thi, tlo);
-        sum += (double)t;
-      }
-    } else {
-      for (int v = lo + threadIdx.x; v < hi; v += kThreads) sum += (double)expo(load1(row, v), M, thi, tlo);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) ss[warp] = sum;
-  __syncthreads();
   pdl_wait();   // the previous step's acceptance may still read the workspace
   if (threadIdx.x == 0) {
     double t = 0.0;
-    for (int w = 0; w < kThreads / 32; ++w) t += ss[w];
+    for (int w = 0; w < kThreads / 32; ++w)
+      if (ss[w] != 0.0) t += sm[w] == M ? ss[w] : ss[w] * exp2(((double)sm[w] - (double)M) * cpow);
     RowStat r;
     r.zm = M;
     r.bi = (M == -INFINITY || Mi == INT_MAX) ? lo : Mi;
@@ -192,7 +204,7 @@ tsd_status launch_accept_threshold(const void* logits, tsd_dtype dtype, int V, c
   if (dtype == TSD_BF16) {
     auto lg = reinterpret_cast<const __nv_bfloat16*>(logits);
     launch_pdl(row_stats_chunks<__nv_bfloat16>, dim3(chunks, Nmax, B), dim3(kThreads), 0, stream, lg, V, Nmax,
-               num_nodes, chunks, thi, tlo, part, vec);
+               num_nodes, chunks, thi, tlo, c, part, vec);
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(tree_threshold_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
@@ -202,7 +214,7 @@ tsd_status launch_accept_threshold(const void* logits, tsd_dtype dtype, int V, c
   } else {
     auto lg = reinterpret_cast<const float*>(logits);
     launch_pdl(row_stats_chunks<float>, dim3(chunks, Nmax, B), dim3(kThreads), 0, stream, lg, V, Nmax, num_nodes,
-               chunks, thi, tlo, part, vec);
+               chunks, thi, tlo, c, part, vec);
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(tree_threshold_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     launch_pdl(tree_threshold_kernel<float>, dim3(B), dim3(kThreads), smem, stream, lg, V, (const RowStat*)part,

@@ -221,10 +221,10 @@ __device__ __forceinline__ int take_ticket(int* word, int splits, int* s_flag) {
 // The last CTA's merge (all threads).  (1) Every split's (max, sum) of every row into shared memory
 // with independent loads; (2) per row the largest split maximum, the splits' weights
 // 2^(M_s - M) / sum (s_w[s][row]) and the log-sum-exp; (3) every (row, 8 columns) the weighted sum
-// of the partial rows, four such pieces per thread and two splits per round so that many loads are
+// of the partial rows, two such pieces per thread and two splits per round so that several loads are
 // in flight, written as bf16.  This CTA's own partial is read from its staged rows in shared memory,
 // the others' from L2 (.cg: written by other SMs).  A split with no mass (M = -inf) has weight 0 and
-// its rows are never used.  Zero rows when the sequence is flagged or out of capacity.
+// its rows are never read.  Zero rows when the sequence is flagged or out of capacity.
 __device__ void merge_splits(const AttnArgs& a, const UParams& u, int b, int g, int G, int r0, int r_hi, int own,
                              bool zero, const uint8_t* sStage, float* s_w, int rows_cap) {
   if (zero) {
@@ -271,10 +271,11 @@ __device__ void merge_splits(const AttnArgs& a, const UParams& u, int b, int g, 
   }
   __syncthreads();
   const int ntask = nrows * (kD / 8);
-  for (int t0 = threadIdx.x; t0 < ntask; t0 += 4 * bd) {
-    float acc[4][8];
+  constexpr int kT = 2;   // pieces per thread per round (registers stay near the main loop's count)
+  for (int t0 = threadIdx.x; t0 < ntask; t0 += kT * bd) {
+    float acc[kT][8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kT; ++j) {
       const int t = t0 + j * bd, cr = t / (kD / 8), c8 = t % (kD / 8);
       const float w = t < ntask ? s_w[own * rows_cap + cr] : 0.f;
       float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
@@ -284,17 +285,14 @@ __device__ void merge_splits(const AttnArgs& a, const UParams& u, int b, int g, 
       }
       acc[j][0] = w * x0.x, acc[j][1] = w * x0.y, acc[j][2] = w * x0.z, acc[j][3] = w * x0.w;
       acc[j][4] = w * x1.x, acc[j][5] = w * x1.y, acc[j][6] = w * x1.z, acc[j][7] = w * x1.w;
-      if (w == 0.f)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
     }
     for (int s0 = 0; s0 < ns; s0 += 2) {
-      float4 x[2][4][2];
+      float4 x[2][kT][2];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int sp = s0 + q;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kT; ++j) {
           const int t = t0 + j * bd, cr = t / (kD / 8), c8 = t % (kD / 8);
           if (sp < ns && sp != own && t < ntask) {
             const float4* p4 = reinterpret_cast<const float4*>(wo + (base + (size_t)sp * u.Rmax + cr) * kD + c8 * 8);
@@ -306,7 +304,7 @@ __device__ void merge_splits(const AttnArgs& a, const UParams& u, int b, int g, 
       for (int q = 0; q < 2; ++q) {
         const int sp = s0 + q;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kT; ++j) {
           const int t = t0 + j * bd, cr = t / (kD / 8);
           if (sp < ns && sp != own && t < ntask) {
             const float w = s_w[sp * rows_cap + cr];
@@ -322,7 +320,7 @@ __device__ void merge_splits(const AttnArgs& a, const UParams& u, int b, int g, 
       }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kT; ++j) {
       const int t = t0 + j * bd, cr = t / (kD / 8), c8 = t % (kD / 8);
       if (t < ntask) {
         const int r = r0 + cr;
