@@ -7,11 +7,11 @@
 // p_parent(i)(token[i]) >= tau; roots, the deepest-node rule and the emitted tokens (the target's
 // own token is the argmax of the last accepted node's row) are those of greedy acceptance.
 //
-// Two launches: a vocabulary scan per (chunk, row) -- the argmax and, relative to the chunk's
-// maximum, the fp64 sum of fp32 exponentials (16-byte loads; the sum re-reads the chunk from
-// cache) -- then one CTA per sequence merges the chunk statistics of every row, decides each
-// edge p >= tau in fp64 from one gathered logit per node, and runs the greedy acceptance walk
-// with those decisions.
+// Two launches: a vocabulary scan per (16384-token chunk, row) -- the argmax and, relative to the
+// chunk's maximum, the fp64 sum of fp32 exponentials in one pass (16-byte loads; a thread's 64
+// logits stay in registers) -- then one CTA per sequence merges the chunk statistics of every row,
+// decides each edge p >= tau in fp64 from one gathered logit per node, and runs the greedy
+// acceptance walk with those decisions.
 #include <climits>
 
 #include "accept_body.cuh"
@@ -23,7 +23,7 @@ namespace tsd {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 8192;
+constexpr int kChunk = 16384;
 constexpr double kLog2eD = 1.4426950408889634074;
 
 struct __align__(16) RowStat {
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kThreads) row_stats_chunks(const T* __restrict
   float wm;          // the warp's maximum: the reference of its exponential sum
   double sum = 0.0;  // the warp's sum relative to wm (lane shares)
   if (vec) {
-    // 16-byte path: the thread's 32 logits of the chunk are loaded at once and stay in registers,
+    // 16-byte path: the thread's 64 logits of the chunk are loaded at once and stay in registers,
     // so the sum is taken relative to the warp's maximum in the same pass
     constexpr int kGroups = kChunk / (kThreads * 8);
     float x[kGroups][8];
@@ -111,17 +111,19 @@ __global__ void __launch_bounds__(kThreads) row_stats_chunks(const T* __restrict
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) sv[warp] = bv, si[warp] = bi, sm[warp] = wm, ss[warp] = sum;
+  if (lane == 0) sv[warp] = bv, si[warp] = bi, sm[warp] = wm;
   __syncthreads();
   float M = -INFINITY;
   int Mi = INT_MAX;
   for (int w = 0; w < kThreads / 32; ++w)
     if (better(sv[w], si[w], M, Mi)) M = sv[w], Mi = si[w];
+  // each warp rescales its own sum to the chunk maximum (fp64, the warps in parallel)
+  if (lane == 0) ss[warp] = (sum == 0.0 || wm == M) ? sum : sum * exp2(((double)wm - (double)M) * cpow);
+  __syncthreads();
   pdl_wait();   // the previous step's acceptance may still read the workspace
   if (threadIdx.x == 0) {
     double t = 0.0;
-    for (int w = 0; w < kThreads / 32; ++w)
-      if (ss[w] != 0.0) t += sm[w] == M ? ss[w] : ss[w] * exp2(((double)sm[w] - (double)M) * cpow);
+    for (int w = 0; w < kThreads / 32; ++w) t += ss[w];
     RowStat r;
     r.zm = M;
     r.bi = (M == -INFINITY || Mi == INT_MAX) ? lo : Mi;

@@ -565,7 +565,9 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
   // the tcgen05 kernel (bf16, d = 128, power-of-two groups) takes two 128-row query tiles per CTA
   // when a KV head has more than 128 query rows, streaming each K/V tile once for both
   const bool umma_shape = dtype == TSD_BF16 && d == 128 && p.G <= 128 && (p.G & (p.G - 1)) == 0;
-  p.dual = umma_shape && p.Rmax > 128;
+  // (TSD_ATTN_DUAL=0 keeps one query tile per CTA: an A/B knob)
+  const char* dual_env = getenv("TSD_ATTN_DUAL");
+  p.dual = umma_shape && p.Rmax > 128 && !(dual_env != nullptr && dual_env[0] == '0');
   p.umtiles = p.dual ? (p.Rmax + 255) / 256 : p.mtiles;
   const long long base = (long long)B * Hkv * (umma_shape ? p.umtiles : p.mtiles);
   const int sms = device_sm_count();

@@ -62,8 +62,10 @@ __device__ __forceinline__ void wtopk_insert(WarpTopK& me, int K, int lane, floa
   }
 }
 
-// Offer each lane's candidate (x, xi) to the warp list; `thr` (the K-th best) is kept current.
-__device__ __forceinline__ void wtopk_offer(WarpTopK& me, WarpTopK& thr, int K, int lane, float x, int xi) {
+// Offer each lane's candidate (x, xi) to the warp list.  `thr` is kept at the larger of the list's
+// K-th best and the floor (floor_v, none): a candidate below it cannot make the top K.
+__device__ __forceinline__ void wtopk_offer(WarpTopK& me, WarpTopK& thr, int K, int lane, float x, int xi,
+                                            float floor_v) {
   unsigned want = __ballot_sync(0xffffffffu, better(x, xi, thr.v, thr.i));
   while (want) {
     const int src = __ffs(want) - 1;
@@ -72,48 +74,41 @@ __device__ __forceinline__ void wtopk_offer(WarpTopK& me, WarpTopK& thr, int K, 
     wtopk_insert(me, K, lane, cx, ci);
     thr.v = __shfl_sync(0xffffffffu, me.v, K - 1);
     thr.i = __shfl_sync(0xffffffffu, me.i, K - 1);
+    if (!better(thr.v, thr.i, floor_v, INT_MAX)) thr.v = floor_v, thr.i = INT_MAX;
     want &= want - 1;
     want &= __ballot_sync(0xffffffffu, better(x, xi, thr.v, thr.i));
   }
 }
 
-// One lane's share of the chunk's exponential sum, kept relative to a reference mt that is the same
-// for the whole warp (the warp's running maximum): st = sum of 2^((x - mt) log2(e)).  When the
-// warp's maximum grows, every lane rescales st by one fp64 exponential (a warp-uniform branch, a few
-// times per chunk), so the only fp32 rounding left is that of each token's own exponential.
-struct LaneSum {
-  float mt = -INFINITY;
-  double st = 0.0;
-};
+// The K-th largest of the 32 lane maxima (ties by lane): at least K tokens of the warp reach it, so
+// it bounds the warp's K-th best from below.  -inf when no lane ranks K-th (NaN maxima).
+__device__ __forceinline__ float kth_lane_max(float lm, int K, int lane) {
+  int rank = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float o = __shfl_sync(0xffffffffu, lm, j);
+    rank += (o > lm || (o == lm && j < lane)) ? 1 : 0;
+  }
+  const unsigned at = __ballot_sync(0xffffffffu, rank == K - 1);
+  const float f = __shfl_sync(0xffffffffu, lm, at ? __ffs(at) - 1 : 0);
+  return at ? f : -INFINITY;
+}
 
 constexpr float kLog2eHi = 1.44269502162933349609375f;            // fp32 part of log2(e)
 constexpr float kLog2eLo = 1.925963033500011079198e-8f;           // log2(e) - kLog2eHi
 
-__device__ __forceinline__ float exp_rel(float x, float mt) {      // e^(x - mt), x <= mt
-  const float d = x - mt;
+__device__ __forceinline__ float exp_rel(float x, float m) {       // e^(x - m), x <= m
+  const float d = x - m;
   return exp2f(fmaf(d, kLog2eHi, d * kLog2eLo));
 }
 
-__device__ __forceinline__ void lane_sum_add8(LaneSum& ls, const float (&x)[8], float m8) {
-  const float wm8 = warp_max(m8);
-  if (wm8 > ls.mt) {
-    if (ls.st != 0.0) ls.st *= exp((double)ls.mt - (double)wm8);
-    ls.mt = wm8;
-  }
-  if (ls.mt == -INFINITY) return;
-  float t = 0.f;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) t += exp_rel(x[e], ls.mt);            // -inf adds 0
-  ls.st += (double)t;
-}
-
 // Offer a group of 8 consecutive tokens (v .. v+7) per lane.  Each lane marks the tokens that reach
-// the warp's K-th best value; while any lane holds a mark, every such lane proposes its first one
-// and the proposals enter the list one at a time (exact comparison, lowest lane first), after which
-// the marks below the new K-th best are dropped.  Late in a chunk a group costs one compare per
-// token and one vote.
+// the threshold (the larger of the warp's K-th best and the floor); while any lane holds a mark,
+// every such lane proposes its first one and the proposals enter the list one at a time (exact
+// comparison, lowest lane first), after which the marks below the new threshold are dropped.  With
+// a good floor a group usually costs one compare per token and one vote.
 __device__ __forceinline__ void offer8(WarpTopK& me, WarpTopK& thr, int K, int lane, const float (&x)[8], int v,
-                                       bool valid) {
+                                       bool valid, float floor_v) {
   unsigned cand = 0;
   if (valid) {
 #pragma unroll
@@ -127,7 +122,7 @@ __device__ __forceinline__ void offer8(WarpTopK& me, WarpTopK& thr, int K, int l
       if (e == j) xv = x[j];
     const int xi = cand ? v + e : INT_MAX;
     cand &= cand - 1;
-    wtopk_offer(me, thr, K, lane, xv, xi);
+    wtopk_offer(me, thr, K, lane, xv, xi, floor_v);
     if (cand) {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
@@ -145,41 +140,50 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpTopK me{-INFINITY, INT_MAX}, thr{-INFINITY, INT_MAX};
-  LaneSum ls;
+  // Pass 1: each lane's maximum; the warp's maximum is the reference of its exponential sum and the
+  // K-th largest lane maximum is the floor of its top-K (at least K tokens reach it).  Pass 2 (the
+  // chunk again, from cache): the exponentials and the offers of the tokens that reach the floor.
+  float lm = -INFINITY;
   if (vec) {
-    // 16-byte loads, the next group in flight while this one is scanned; every lane of a warp
-    // runs the same trips (a lane past the end offers nothing)
-    float x[8], y[8];
-    int v = lo + threadIdx.x * 8;
-    if (v < hi) load8<T>(row, v, x);
-#pragma unroll 1
-    for (; v - threadIdx.x * 8 < hi; v += kThreads * 8) {
+    for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
+      float x[8];
+      load8<T>(row, v, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[e]);
+    }
+  } else {
+    for (int v = lo + threadIdx.x; v < hi; v += kThreads) lm = fmaxf(lm, load1(row, v));
+  }
+  const float wm = warp_max(lm);
+  const float floor_v = kth_lane_max(lm, K, lane);
+  thr.v = floor_v;
+  double wsum = 0.0;
+  if (vec) {
+    // every lane of a warp runs the same trips (a lane past the end offers nothing)
+    for (int g0 = lo; g0 < hi; g0 += kThreads * 8) {
+      const int v = g0 + threadIdx.x * 8;
       const bool valid = v < hi;
-      const int vn = v + kThreads * 8;
-      if (vn < hi) load8<T>(row, vn, y);
-      if (!valid) {
+      float x[8];
+      if (valid) {
+        load8<T>(row, v, x);
+      } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = -INFINITY;
       }
-      float m8 = x[0];
+      if (wm != -INFINITY) {
+        float t = 0.f;
 #pragma unroll
-      for (int e = 1; e < 8; ++e) m8 = fmaxf(m8, x[e]);
-      offer8(me, thr, K, lane, x, v, valid);
-      lane_sum_add8(ls, x, m8);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = y[e];
+        for (int e = 0; e < 8; ++e) t += exp_rel(x[e], wm);   // -inf adds 0
+        wsum += (double)t;
+      }
+      offer8(me, thr, K, lane, x, v, valid, floor_v);
     }
   } else {
     for (int v0 = lo; v0 < hi; v0 += kThreads) {
       const int v = v0 + threadIdx.x;
       const float x = v < hi ? load1(row, v) : -INFINITY;
-      wtopk_offer(me, thr, K, lane, x, v < hi ? v : INT_MAX);
-      const float wx = warp_max(x);
-      if (wx > ls.mt) {
-        if (ls.st != 0.0) ls.st *= exp((double)ls.mt - (double)wx);
-        ls.mt = wx;
-      }
-      if (ls.mt != -INFINITY) ls.st += (double)exp_rel(x, ls.mt);
+      if (wm != -INFINITY) wsum += (double)exp_rel(x, wm);
+      wtopk_offer(me, thr, K, lane, x, v < hi ? v : INT_MAX, floor_v);
     }
   }
   // chunk maximum and sum: the warps' sums (relative to their maxima), then the block's maximum
@@ -187,8 +191,7 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
   __shared__ double s_s[kThreads / 32];
   __shared__ float s_wv[kThreads / 32][kMaxK];
   __shared__ int s_wi[kThreads / 32][kMaxK];
-  const float wm = ls.mt;   // the same in every lane
-  double sum = ls.st;
+  double sum = wsum;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (lane == 0) s_m[warp] = wm, s_s[warp] = sum;
