@@ -690,14 +690,18 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       const int k = kDual ? i : i >> 1;            // this warpgroup's k-th tile
       const int buf = kDual ? wg : wg + 2 * (k & 1);
       const uint32_t s_col = kColS + (uint32_t)buf * kBN;
-      if (!mbar_wait(&bars.s_full[buf], kDual ? (k & 1) : ((k >> 1) & 1), u.wait)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
       const int t = t_begin + i;
       const bool tree = t >= v.nPT;
       const int kbase = tree ? (t - v.nPT) * kBN : t * kBN;
+      if (ok && !mbar_wait(&bars.s_full[buf], kDual ? (k & 1) : ((k >> 1) & 1), u.wait)) ok = false;
+      if (ok && tree && !mask_ready) {
+        if (mbar_wait(&bars.mask_full, 0, u.wait)) mask_ready = true;
+        else ok = false;
+      }
+      // one verdict per warp: the TMEM accesses below are warp-collective
+      ok = __all_sync(0xffffffffu, ok) != 0;
+      if (!ok) break;
+      tc_fence_after();
       float alpha = 1.f;
       bool resc = false;
       uint32_t pk[32];
@@ -720,13 +724,6 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         } else {
           const int lim = tree ? v.N : v.L;
           uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
-          if (tree && !mask_ready) {
-            if (!mbar_wait(&bars.mask_full, 0, u.wait)) {
-              ok = false;
-              break;
-            }
-            mask_ready = true;
-          }
           if (tree) {
             const int wi = kbase >> 5;
             w0 = sMask[nl * u.W + wi];
@@ -789,8 +786,10 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         }
         l = l * alpha + ((suma[0] + suma[1]) + (suma[2] + suma[3]));
       }
-      // this warpgroup's previous P V (tile i - 2) must be done before O is rescaled
-      if (k >= 1 && !mbar_wait(&bars.pv_done[wg], (k - 1) & 1, u.wait)) {
+      // this warpgroup's previous P V must be done before O is rescaled (one verdict per warp: the
+      // TMEM accesses below are warp-collective)
+      bool pv_ok = k < 1 || mbar_wait(&bars.pv_done[wg], (k - 1) & 1, u.wait);
+      if (!__all_sync(0xffffffffu, pv_ok)) {
         ok = false;
         break;
       }
