@@ -206,6 +206,33 @@ def test_chain_sample_small(V, dt):
     assert np.array_equal(got["out_tokens"], ref["out_tokens"])
 
 
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_chain_sample_masked_vocabulary(dt):
+    """-inf logits (a masked vocabulary, 30% of the tokens) in every target and draft row, at
+    T = 0.7 (an exponent constant whose fp32 split has a negative low part) and T = 1: the masked
+    tokens carry no mass, are never emitted, and every decision is the oracle's."""
+    rng = np.random.default_rng(23)
+    B, K, V = 128, 4, 4096
+    zpf = rng.standard_normal((B, K + 1, V)).astype(np.float32) * 2
+    zqf = zpf[:, :K] + rng.standard_normal((B, K, V)).astype(np.float32) * 0.8
+    masked = rng.random(V) < 0.3
+    zpf[..., masked] = -np.inf
+    zqf[..., masked] = -np.inf
+    zp = W.f32_to_bf16_bits(zpf) if dt == "bf16" else zpf
+    zq = W.f32_to_bf16_bits(zqf) if dt == "bf16" else zqf
+    open_ids = np.nonzero(~masked)[0]
+    x = open_ids[rng.integers(0, len(open_ids), size=(B, K))].astype(np.int32)
+    am = W.as_f32(zq, dt).argmax(-1)
+    x = np.where(rng.random((B, K)) < 0.7, am, x).astype(np.int32)
+    u = rng.random((B, K + 1), dtype=np.float32)
+    for T in (0.7, 1.0):
+        got = gpu_sample(zp, zq, x, u, T)
+        ref = oracle.chain_sample(zp, zq, x, u, T)
+        assert compare_sampling(got, ref, K, zp, zq, u, T, x) <= 3
+        emitted = got["out_tokens"][got["out_tokens"] >= 0]
+        assert not masked[emitted].any()
+
+
 def test_chain_sample_distribution_gpu():
     """The GPU sampler preserves the target distribution (chi-square, vocab 16, K = 3, toy
     Markov target and draft as in the oracle's own distribution test)."""

@@ -54,18 +54,19 @@ __global__ void __launch_bounds__(kThreads) row_stats_chunks(const T* __restrict
   const T* row = logits + ((size_t)b * rows_per_seq + i) * V;
   const int lo = c * kChunk, hi = min(V, lo + kChunk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __shared__ float sv[kThreads / 32], sm[kThreads / 32];
+  __shared__ float sm[kThreads / 32];
   __shared__ int si[kThreads / 32];
   __shared__ double ss[kThreads / 32];
-  float bv = -INFINITY;
-  int bi = INT_MAX;
-  float wm;          // the warp's maximum: the reference of its exponential sum
-  double sum = 0.0;  // the warp's sum relative to wm (lane shares)
+  float lm = -INFINITY;   // the lane's maximum
+  int li = INT_MAX;       // its lowest index (one-element path; the 16-byte path finds it on demand)
+  double sum = 0.0;       // the lane's share of the chunk sum, relative to the warp's maximum
+  constexpr int kGroups = kChunk / (kThreads * 8);
+  float x[kGroups][8];
+  float wm;
   if (vec) {
-    // 16-byte path: the thread's 64 logits of the chunk are loaded at once and stay in registers,
-    // so the sum is taken relative to the warp's maximum in the same pass
-    constexpr int kGroups = kChunk / (kThreads * 8);
-    float x[kGroups][8];
+    // 16-byte path: the thread's 64 logits of the chunk are loaded at once and stay in registers:
+    // the maximum, then the exponentials relative to the warp's maximum (paired instructions), and
+    // the argmax index searched only by the lanes holding the chunk's maximum
 #pragma unroll
     for (int gi = 0; gi < kGroups; ++gi) {
       const int v = lo + (gi * kThreads + threadIdx.x) * 8;
@@ -77,53 +78,56 @@ __global__ void __launch_bounds__(kThreads) row_stats_chunks(const T* __restrict
       }
     }
 #pragma unroll
-    for (int gi = 0; gi < kGroups; ++gi) {
-      const int v = lo + (gi * kThreads + threadIdx.x) * 8;
+    for (int gi = 0; gi < kGroups; ++gi)
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (x[gi][e] > bv) bv = x[gi][e], bi = v + e;   // ascending order: ties keep the lower index
-    }
-    wm = warp_max(bv);
-    if (wm != -INFINITY) {
+      for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[gi][e]);
+    wm = warp_max(lm);
+    if (wm != -INFINITY)
 #pragma unroll
-      for (int gi = 0; gi < kGroups; ++gi) {
-        float t = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t += expo(x[gi][e], wm, thi, tlo);   // -inf adds 0
-        sum += (double)t;
-      }
-    }
+      for (int gi = 0; gi < kGroups; ++gi) sum += (double)sum_ex2_8(x[gi], wm, thi, tlo);
   } else {
     for (int v = lo + threadIdx.x; v < hi; v += kThreads) {
-      const float x = load1(row, v);
-      if (better(x, v, bv, bi)) bv = x, bi = v;
+      const float xv = load1(row, v);
+      if (better(xv, v, lm, li)) lm = xv, li = v;
     }
-    wm = warp_max(bv);
+    wm = warp_max(lm);
     if (wm != -INFINITY)
       for (int v = lo + threadIdx.x; v < hi; v += kThreads) sum += (double)expo(load1(row, v), wm, thi, tlo);
   }
-  // block argmax (ties -> lower index) and maximum; the warps' sums rescaled to it in fp64
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (better(ov, oi, bv, bi)) bv = ov, bi = oi;
-  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) sv[warp] = bv, si[warp] = bi, sm[warp] = wm;
+  if (lane == 0) sm[warp] = wm;
   __syncthreads();
   float M = -INFINITY;
-  int Mi = INT_MAX;
-  for (int w = 0; w < kThreads / 32; ++w)
-    if (better(sv[w], si[w], M, Mi)) M = sv[w], Mi = si[w];
+  for (int w = 0; w < kThreads / 32; ++w) M = fmaxf(M, sm[w]);
+  // the lowest index holding the chunk maximum (ties -> lower index)
+  int idx = INT_MAX;
+  if (M != -INFINITY && lm == M) {
+    if (vec) {
+#pragma unroll
+      for (int gi = kGroups - 1; gi >= 0; --gi) {
+        const int v = lo + (gi * kThreads + threadIdx.x) * 8;
+#pragma unroll
+        for (int e = 7; e >= 0; --e)
+          if (x[gi][e] == M) idx = v + e;
+      }
+    } else {
+      idx = li;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) idx = min(idx, __shfl_xor_sync(0xffffffffu, idx, o));
   // each warp rescales its own sum to the chunk maximum (fp64, the warps in parallel)
-  if (lane == 0) ss[warp] = (sum == 0.0 || wm == M) ? sum : sum * exp2(((double)wm - (double)M) * cpow);
+  if (lane == 0) {
+    si[warp] = idx;
+    ss[warp] = (sum == 0.0 || wm == M) ? sum : sum * exp2(((double)wm - (double)M) * cpow);
+  }
   __syncthreads();
   pdl_wait();   // the previous step's acceptance may still read the workspace
   if (threadIdx.x == 0) {
     double t = 0.0;
-    for (int w = 0; w < kThreads / 32; ++w) t += ss[w];
+    int Mi = INT_MAX;
+    for (int w = 0; w < kThreads / 32; ++w) t += ss[w], Mi = min(Mi, si[w]);
     RowStat r;
     r.zm = M;
     r.bi = (M == -INFINITY || Mi == INT_MAX) ? lo : Mi;
@@ -199,7 +203,8 @@ tsd_status launch_accept_threshold(const void* logits, tsd_dtype dtype, int V, c
   if (B == 0) return TSD_OK;
   const int chunks = num_chunks(V);
   const double c = kLog2eD / (double)T;
-  const float thi = (float)c, tlo = (float)(c - (double)thi);
+  float thi, tlo;
+  split_const(c, thi, tlo);
   RowStat* part = reinterpret_cast<RowStat*>(ws);
   const int vec = vec16_rows(logits, V) ? 1 : 0;
   const size_t smem = accept_threshold_smem(Nmax);

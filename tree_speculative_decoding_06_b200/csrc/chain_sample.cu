@@ -114,39 +114,50 @@ __global__ void __launch_bounds__(kThreads) chain_stats(const T* __restrict__ zp
   __shared__ float sm[kThreads / 32];
   __shared__ double sd[kThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float mx = -INFINITY;
+  // one read of the chunk: a thread's 32 logits stay in registers (16-byte path); each warp sums
+  // its exponentials relative to its own maximum, then the warps' sums are rescaled (fp64) to the
+  // chunk maximum
+  float lm = -INFINITY, wm;
+  double s = 0.0;
   if (vec) {
-    for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
-      float x[8];
-      load8<T>(row, v, x);
+    constexpr int kGroups = kChunk / (kThreads * 8);
+    float x[kGroups][8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx = fmaxf(mx, x[e]);
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int v = lo + (gi * kThreads + threadIdx.x) * 8;
+      if (v < hi) {
+        load8<T>(row, v, x[gi]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[gi][e] = -INFINITY;
+      }
     }
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[gi][e]);
+    wm = warp_max(lm);
+    if (wm != -INFINITY)
+#pragma unroll
+      for (int gi = 0; gi < kGroups; ++gi) s += (double)sum_exp2f_8(x[gi], wm, tc.hi, tc.lo);   // -inf adds 0
   } else {
-    for (int v = lo + threadIdx.x; v < hi; v += kThreads) mx = fmaxf(mx, load1(row, v));
+    for (int v = lo + threadIdx.x; v < hi; v += kThreads) lm = fmaxf(lm, load1(row, v));
+    wm = warp_max(lm);
+    if (wm != -INFINITY)
+      for (int v = lo + threadIdx.x; v < hi; v += kThreads) s += (double)expo(load1(row, v), wm, tc);
   }
-  mx = warp_max(mx);
-  if (lane == 0) sm[warp] = mx;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) sm[warp] = wm;
   __syncthreads();
   float zm = -INFINITY;
 #pragma unroll
   for (int w = 0; w < kThreads / 32; ++w) zm = fmaxf(zm, sm[w]);
-  double s = 0.0;
-  if (zm != -INFINITY) {
-    if (vec) {
-      for (int v = lo + threadIdx.x * 8; v < hi; v += kThreads * 8) {
-        float x[8];
-        load8<T>(row, v, x);
-        float t = 0.f;
+  if (lane == 0) sd[warp] = (s == 0.0 || wm == zm) ? s : s * exp2(((double)wm - (double)zm) * tc.c);
+  __syncthreads();
+  s = 0.0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t += expo(x[e], zm, tc);
-        s += (double)t;
-      }
-    } else {
-      for (int v = lo + threadIdx.x; v < hi; v += kThreads) s += (double)expo(load1(row, v), zm, tc);
-    }
-  }
-  s = block_sum_d(s, sd);
+  for (int w = 0; w < kThreads / 32; ++w) s += sd[w];
   pdl_wait();
   if (threadIdx.x == 0) {
     Stat st;
@@ -368,8 +379,7 @@ tsd_status launch_chain_sample_stochastic(const void* zp, const void* zq, tsd_dt
   double* mass = reinterpret_cast<double*>(fin + B);
   Temp tc;
   tc.c = kLog2eD / (double)T;
-  tc.hi = (float)tc.c;
-  tc.lo = (float)(tc.c - (double)tc.hi);
+  split_const(tc.c, tc.hi, tc.lo);
   const size_t dsmem = (size_t)(2 * K + 1) * sizeof(Stat) + (size_t)2 * K * sizeof(float) + 16;
   dim3 g1(chunks, 2 * K + 1, B), g3(chunks, B);
   const int vec = vec16_rows(zp, V) && (K == 0 || vec16_rows(zq, V)) ? 1 : 0;

@@ -45,6 +45,59 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
+// Paired fp32 arithmetic of sm_100 (two lanes of work per instruction), round to nearest.
+__device__ __forceinline__ void padd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n.reg .b64 ra, rb, rd;\nmov.b64 ra, {%2, %3};\nmov.b64 rb, {%4, %5};\n"
+      "add.rn.f32x2 rd, ra, rb;\nmov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void pmul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n.reg .b64 ra, rb, rd;\nmov.b64 ra, {%2, %3};\nmov.b64 rb, {%4, %5};\n"
+      "mul.rn.f32x2 rd, ra, rb;\nmov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void pfma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0, float c1) {
+  asm("{\n.reg .b64 ra, rb, rc, rd;\nmov.b64 ra, {%2, %3};\nmov.b64 rb, {%4, %5};\nmov.b64 rc, {%6, %7};\n"
+      "fma.rn.f32x2 rd, ra, rb, rc;\nmov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+// 2^x by the hardware approximation, results below 2^-126 flushed to zero (a sum whose largest term
+// is 1 does not see them); 2^-inf = 0.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+// sum over e of 2^((x[e] - m) * (chi + clo)) for 8 values x[e] <= m: x - m in one rounding (exact
+// for bf16 logits), the two-term constant applied as d*chi + d*clo, paired instructions.
+__device__ __forceinline__ float sum_ex2_8(const float (&x)[8], float m, float chi, float clo) {
+  float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    float d0, d1, u0, u1, a0, a1;
+    padd2(d0, d1, x[e], x[e + 1], -m, -m);
+    pmul2(u0, u1, d0, d1, clo, clo);
+    pfma2(a0, a1, d0, d1, chi, chi, u0, u1);
+    padd2(t0, t1, t0, t1, ex2_ftz(a0), ex2_ftz(a1));
+  }
+  return t0 + t1;
+}
+
+// The same sum with the library exp2f for each term (its accuracy where a sampler's decisions are
+// compared with an fp64 oracle at tight margins).
+__device__ __forceinline__ float sum_exp2f_8(const float (&x)[8], float m, float chi, float clo) {
+  float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    float d0, d1, u0, u1, a0, a1;
+    padd2(d0, d1, x[e], x[e + 1], -m, -m);
+    pmul2(u0, u1, d0, d1, clo, clo);
+    pfma2(a0, a1, d0, d1, chi, chi, u0, u1);
+    padd2(t0, t1, t0, t1, exp2f(a0), exp2f(a1));
+  }
+  return t0 + t1;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

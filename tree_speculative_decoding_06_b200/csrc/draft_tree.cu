@@ -109,8 +109,11 @@ __device__ __forceinline__ float exp_rel(float x, float m) {       // e^(x - m),
 // a good floor a group usually costs one compare per token and one vote.
 __device__ __forceinline__ void offer8(WarpTopK& me, WarpTopK& thr, int K, int lane, const float (&x)[8], int v,
                                        bool valid, float floor_v) {
+  float m8 = x[0];
+#pragma unroll
+  for (int e = 1; e < 8; ++e) m8 = fmaxf(m8, x[e]);
   unsigned cand = 0;
-  if (valid) {
+  if (valid && m8 >= thr.v) {   // usually not: the floor dismisses the whole group
 #pragma unroll
     for (int e = 0; e < 8; ++e) cand |= (x[e] >= thr.v ? 1u : 0u) << e;
   }
@@ -170,12 +173,7 @@ __global__ void __launch_bounds__(kThreads) draft_row_stats(const T* __restrict_
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = -INFINITY;
       }
-      if (wm != -INFINITY) {
-        float t = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t += exp_rel(x[e], wm);   // -inf adds 0
-        wsum += (double)t;
-      }
+      if (wm != -INFINITY) wsum += (double)sum_ex2_8(x, wm, kLog2eHi, kLog2eLo);   // -inf adds 0
       offer8(me, thr, K, lane, x, v, valid, floor_v);
     }
   } else {

@@ -1,6 +1,7 @@
 // Internal launch entry points of the kernels (host side); the C ABI in api.cu validates
 // arguments and calls these.
 #pragma once
+#include <cmath>
 
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -20,6 +21,16 @@ inline bool vec16_rows(const void* base, int V) {
   return V % 8 == 0 && (reinterpret_cast<uintptr_t>(base) & 15) == 0;
 }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// A positive constant c as an unevaluated sum hi + lo of floats with lo > 0 (hi rounded toward
+// zero; a tiny lo when c is itself a float), so that d * hi + d * lo is -inf, not -inf + inf, for
+// d = -inf (a -inf logit, or -inf padding).
+inline void split_const(double c, float& hi, float& lo) {
+  hi = (float)c;
+  if ((double)hi > c) hi = std::nextafter(hi, 0.0f);
+  lo = (float)(c - (double)hi);
+  if (!(lo > 0.f)) lo = 1e-30f;
+}
 
 // Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger in common.cuh).
 template <typename... KArgs, typename... Args>

@@ -468,8 +468,7 @@ tsd_status launch_ssd_cache(const void* zq, tsd_dtype dtype, int V, int K, int S
   SSDArgs a{};
   a.zq = zq, a.V = V, a.K = K, a.S = S, a.alpha = alpha, a.beta = beta, a.u = u;
   const double c = kLog2eD / (double)T;
-  a.thi = (float)c;
-  a.tlo = (float)(c - (double)a.thi);
+  split_const(c, a.thi, a.tlo);
   a.slice = ((V + kC - 1) / kC + 7) / 8 * 8;
   a.vec = vec16_rows(zq, V) ? 1 : 0;
   a.slots = slots, a.key_len = key_len, a.key_tok = key_tok, a.draft_tokens = draft_tokens;

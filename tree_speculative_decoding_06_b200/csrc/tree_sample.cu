@@ -490,8 +490,7 @@ tsd_status launch_tree_sample(const void* zp, const void* zq, tsd_dtype dtype, i
   TSArgs a{};
   a.zp = zp, a.zq = zq, a.V = V, a.tokens = tokens, a.parent_s = parent_s, a.num_nodes = num_nodes, a.u = u;
   const double c = kLog2eD / (double)T;
-  a.tc.hi = (float)c;
-  a.tc.lo = (float)(c - (double)a.tc.hi);
+  split_const(c, a.tc.hi, a.tc.lo);
   a.Nmax = Nmax, a.Dmax = Dmax;
   a.slice = ((V + kC - 1) / kC + 7) / 8 * 8;
   a.vec = vec16_rows(zp, V) && vec16_rows(zq, V) ? 1 : 0;
