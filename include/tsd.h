@@ -168,6 +168,14 @@ size_t tsd_tree_verify_attn_workspace_size(int B, int Nmax, int Hq, int Hkv, int
 /* Size of the ticket region at the start of an attention workspace (a constant). */
 size_t tsd_tree_verify_attn_ticket_bytes(void);
 
+/* Number of kernels one tsd_tree_verify_attn[_paged] call launches on its stream for these sizes
+ * (1: the split kernel alone, its key splits merged inside it or not split; 2: followed by the
+ * merge kernel), for 16-byte-aligned tensors and a workspace of the queried size.  Lmax is the
+ * capacity (max_blocks * block_size for the paged call), block_size 0 for the contiguous cache,
+ * tree_in_cache 1 when k_tree / v_tree are NULL.  A host function; 0 for invalid sizes. */
+int tsd_tree_verify_attn_kernels(int B, int Nmax, int Hq, int Hkv, int d, int Lmax, int block_size, int tree_in_cache,
+                                 tsd_dtype dtype);
+
 tsd_status tsd_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache, int Lmax,
                                 const int32_t *prefix_len, const void *k_tree, const void *v_tree,
                                 const int32_t *parent_s, const int32_t *num_nodes, int B, int Nmax, int Hq,

@@ -104,12 +104,13 @@ def test_host_checks_of_the_fused_and_draft_tree_entry_points():
 def test_split_planner_choices_for_the_bench_workloads():
     """The planner's split counts (read back through the workspace size: splits * rows * (d + 2)
     fp32 per KV head and sequence) for the four bench shapes on a 148-SM device: tree26 9 (a sweep
-    of 3..17 on B200 found 9 fastest), eagle60 3 (paged: planned for ragged lengths, each split an
-    equal share of its own sequence, longest sequences first), chain5 2, forest 2."""
+    of 3..17 on B200 found 9 fastest), eagle60 2 (paged: planned for ragged lengths, each split an
+    equal share of its own sequence, longest sequences first; a B200 sweep of 2..8 found 2 fastest
+    with the splits merged in the kernel), chain5 2, forest 2 (a sweep of 1..4: 2)."""
     def splits(ws, B, Hkv, R, d=128):   # the ticket words come first, then the partials
         return (ws - tsd.tree_verify_attn_ticket_bytes()) // (B * Hkv * R * (d + 2) * 4) if ws else 1
     assert splits(tsd.tree_verify_attn_workspace_size(1, 26, 32, 8, 128, 2112, 1), 1, 8, 104) == 9
-    assert splits(tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1), 16, 8, 240) == 3
+    assert splits(tsd.tree_verify_attn_paged_workspace_size(16, 60, 32, 8, 128, 520, 16, 1), 16, 8, 240) == 2
     assert splits(tsd.tree_verify_attn_workspace_size(64, 6, 64, 8, 128, 8256, 1), 64, 8, 48) == 2
     assert splits(tsd.tree_verify_attn_paged_workspace_size(8, 512, 32, 8, 128, 2080, 16, 1), 8, 8, 2048) == 2
 
@@ -138,3 +139,23 @@ def test_misaligned_tensor_pointers_are_refused_before_any_launch():
     need = tsd.tree_accept_greedy_workspace_size(1, 4, 64)
     assert L.tsd_tree_accept_greedy(p, 1, 64, p, p, None, None, 1, 4, 3, p, p, p, odd, need, p, None) == 9
     assert tsd.accept_noalloc_scratch_bytes() == 1 << 20
+
+
+def test_attention_kernel_count_query(monkeypatch):
+    """Kernels per attention call, as the bench counts them: the two-tile tcgen05 kernel merges its
+    key splits itself (eagle60, forest: one launch), the one-tile kernel (tree26, chain5) and the
+    mma.sync path are followed by the merge kernel; TSD_ATTN_MERGE forces either merge."""
+    monkeypatch.delenv("TSD_ATTN_MERGE", raising=False)
+    monkeypatch.delenv("TSD_ATTN_PATH", raising=False)
+    q = tsd.tree_verify_attn_kernels
+    assert q(1, 26, 32, 8, 128, 2112, 1) == 2                    # tree26: 9 splits, merge kernel
+    assert q(16, 60, 32, 8, 128, 520 * 16, 1, 16) == 1           # eagle60 (paged): merged in the kernel
+    assert q(64, 6, 64, 8, 128, 8256, 1) == 2                    # chain5
+    assert q(8, 512, 32, 8, 128, 2080 * 16, 1, 16) == 1          # forest (paged)
+    assert q(1, 8, 8, 2, 64, 128, 0) in (1, 2)                   # fp32 FFMA path
+    assert q(16, 60, 32, 8, 128, 8320, 1, 0, True) in (1, 2)     # tree K/V in the cache: mma.sync path
+    monkeypatch.setenv("TSD_ATTN_MERGE", "kernel")
+    assert q(16, 60, 32, 8, 128, 520 * 16, 1, 16) == 2
+    monkeypatch.setenv("TSD_ATTN_MERGE", "fused")
+    assert q(1, 26, 32, 8, 128, 2112, 1) == 1
+    assert q(0, 26, 32, 8, 128, 2112, 1) == 0

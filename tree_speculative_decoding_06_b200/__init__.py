@@ -40,6 +40,7 @@ _SIGS = {
                                   _P, _SZ, _P, _P]),
     "tsd_tree_verify_attn_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "tsd_tree_verify_attn_ticket_bytes": (_SZ, []),
+    "tsd_tree_verify_attn_kernels": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "tsd_tree_verify_attn_paged": (_I, [_P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                         _I, _F, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_accept_greedy_workspace_size": (_SZ, [_I, _I, _I]),
@@ -169,6 +170,12 @@ def tree_verify_attn_paged_workspace_size(B, Nmax, Hq, Hkv, d, max_blocks, block
 def tree_verify_attn_ticket_bytes() -> int:
     """Bytes of split-merge ticket words at the start of an attention workspace (kept zero)."""
     return int(lib().tsd_tree_verify_attn_ticket_bytes())
+
+
+def tree_verify_attn_kernels(B, Nmax, Hq, Hkv, d, Lmax, dtype, block_size: int = 0, tree_in_cache: bool = False) -> int:
+    """Kernels one attention call launches for these sizes (the split kernel, and the merge kernel
+    when the keys are split and not merged inside it); Lmax = capacity, block_size 0 = contiguous."""
+    return int(lib().tsd_tree_verify_attn_kernels(B, Nmax, Hq, Hkv, d, Lmax, block_size, int(tree_in_cache), dtype))
 
 
 def _nbytes(ws) -> int:

@@ -602,13 +602,16 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
   // CTA and the total work over the SMs).  Each split adds partials to write and merge.
   if (umma_shape) {
     const long long ubase = (long long)B * Hkv * p.umtiles;
+    // a two-tile CTA's fixed cost (Q rows into TMEM, the first K/V tiles through the block table,
+    // the epilogue and the in-kernel merge) measured ~8 key tiles; a one-tile CTA's ~2
+    const double uover = p.dual ? 8.0 : overhead;
     double best = 1e300;
     for (int c = 1; c <= 32; ++c) {
-      const double per = (double)((p.max_tiles + c - 1) / c) + overhead;
+      const double per = (double)((p.max_tiles + c - 1) / c) + uover;
       const double waves = (double)((ubase * c + sms - 1) / sms);
       double cost = waves * per;
       if (paged) {
-        const double spread = fmax(per, (double)ubase * (0.5 * p.max_tiles + c * overhead) / sms);
+        const double spread = fmax(per, (double)ubase * (0.5 * p.max_tiles + c * uover) / sms);
         cost = 0.5 * (cost + spread);
       }
       cost += c > 1 ? 0.35 * c : 0.0;
@@ -618,6 +621,23 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
   const int wsplits = p.splits > p.usplits ? p.splits : p.usplits;   // either kernel may run
   p.ws_bytes = wsplits > 1 ? kAttnTicketBytes + (size_t)B * Hkv * wsplits * p.Rmax * (d + 2) * sizeof(float) : 0;
   return p;
+}
+
+int attention_launch_count(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype, bool paged,
+                           bool tree_in_cache) {
+  if (B <= 0 || Nmax <= 0 || Hkv <= 0) return 0;
+  const AttnPlan p = plan_attention(B, Nmax, Hq, Hkv, d, Lcap, dtype, paged);
+  const char* path_env = getenv("TSD_ATTN_PATH");
+  const bool force_mma = path_env != nullptr && path_env[0] == 'm' && path_env[1] == 'm';
+  const int G = Hq / Hkv;
+  // the tcgen05 kernel's conditions (umma_eligible), for aligned tensors
+  const bool umma = dtype == TSD_BF16 && d == 128 && !tree_in_cache && G >= 1 && G <= 128 && (G & (G - 1)) == 0 &&
+                    Lcap > 0 && !force_mma;
+  if (!umma) return p.splits > 1 ? 2 : 1;
+  if (p.usplits <= 1) return 1;
+  UmmaLayout L;
+  if (!umma_layout(p, G, Nmax, L)) return 0;
+  return umma_merges_in_kernel(p, L, B, Hkv) ? 1 : 2;
 }
 
 tsd_status launch_attention(const AttnArgs& a_in, tsd_dtype dtype, cudaStream_t stream) {

@@ -1009,6 +1009,45 @@ bool umma_eligible(const AttnArgs& a, tsd_dtype dtype) {
   return encoder() != nullptr;
 }
 
+bool umma_layout(const AttnPlan& p, int G, int Nmax, UmmaLayout& L) {
+  L.rows = p.dual ? 2 * kBM : kBM;                     // query rows per CTA
+  const uint32_t q_bytes = p.dual ? 0u : kQBytes;      // two query tiles live in TMEM, not shared memory
+  L.W = (Nmax + 31) / 32;
+  const uint32_t mask_bytes = (uint32_t)(L.rows / G) * L.W * 4;
+  const uint32_t ps_bytes = (uint32_t)(Nmax + 1) * 4;   // the tree's parent slots, staged for the mask
+  auto total = [&](int ks, int vs) {
+    return 1024 + q_bytes + (uint32_t)(ks + vs) * kSlot + ((mask_bytes + 15) & ~15u) + ps_bytes;
+  };
+  L.ks = 6, L.vs = 5;   // K is consumed first (by S = Q K^T), so its ring runs further ahead
+  const uint32_t limit = 227 * 1024 - 4096;   // leave room for the static shared variables
+  while (total(L.ks, L.vs) > limit && L.vs > 2) {
+    if (L.ks > L.vs) --L.ks; else --L.vs;
+  }
+  if (total(L.ks, L.vs) > limit) return false;
+  L.k_off = q_bytes;
+  L.v_off = L.k_off + (uint32_t)L.ks * kSlot;
+  L.mask_off = L.v_off + (uint32_t)L.vs * kSlot;
+  L.ps_off = L.mask_off + ((mask_bytes + 15) & ~15u);
+  L.stage = (uint32_t)(L.ks + L.vs) * kSlot >= (uint32_t)L.rows * kStageF ? 1 : 0;
+  L.smem = total(L.ks, L.vs);
+  return true;
+}
+
+// Split merge in the kernel: the last CTA's staged rows and the splits' weights fit in the rings,
+// and the ticket words fit their region.  Measured on B200: it pays for the two-tile kernel (256
+// rows per CTA: the merge kernel re-reads large partials from DRAM after the grid ends), not for
+// one-tile CTAs (many short CTAs pay the fence and ticket round trips; many splits leave one CTA a
+// long merge), which keep the merge kernel.  TSD_ATTN_MERGE=kernel / =fused force either choice
+// (A/B runs).
+bool umma_merges_in_kernel(const AttnPlan& p, const UmmaLayout& L, int B, int Hkv) {
+  const char* merge_env = getenv("TSD_ATTN_MERGE");
+  const long long groups = (long long)B * Hkv * p.umtiles;
+  const bool want = merge_env != nullptr ? merge_env[0] == 'f' : p.dual;
+  return want && p.usplits > 1 && L.stage &&
+         (size_t)(L.ks + L.vs) * kSlot >= (size_t)L.rows * kStageF + (size_t)p.usplits * L.rows * 12 &&
+         groups * 4 <= (long long)kAttnTicketBytes;
+}
+
 tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, int* tickets, bool* merged,
                                  cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
@@ -1024,40 +1063,14 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, int* tick
     u.withhold = atoi(w);
     u.wait = 100000;
   }
-  const int rows = p.dual ? 2 * kBM : kBM;   // query rows per CTA
-  const uint32_t q_bytes = p.dual ? 0u : kQBytes;   // two query tiles live in TMEM, not shared memory
-  u.W = (a.Nmax + 31) / 32;
-  const uint32_t mask_bytes = (uint32_t)(rows / G) * u.W * 4;
-  const uint32_t ps_bytes = (uint32_t)(a.Nmax + 1) * 4;   // the tree's parent slots, staged for the mask
-  auto total = [&](int ks, int vs) {
-    return 1024 + q_bytes + (uint32_t)(ks + vs) * kSlot + ((mask_bytes + 15) & ~15u) + ps_bytes;
-  };
-  u.ks = 6, u.vs = 5;   // K is consumed first (by S = Q K^T), so its ring runs further ahead
-  const uint32_t limit = 227 * 1024 - 4096;   // leave room for the static shared variables
-  while (total(u.ks, u.vs) > limit && u.vs > 2) {
-    if (u.ks > u.vs) --u.ks; else --u.vs;
-  }
-  if (total(u.ks, u.vs) > limit) return TSD_ERR_INVALID_ARG;
-  u.k_off = q_bytes;
-  u.v_off = u.k_off + (uint32_t)u.ks * kSlot;
-  u.mask_off = u.v_off + (uint32_t)u.vs * kSlot;
-  u.ps_off = u.mask_off + ((mask_bytes + 15) & ~15u);
-  u.stage = (uint32_t)(u.ks + u.vs) * kSlot >= (uint32_t)rows * kStageF ? 1 : 0;
-  // split merge in the kernel: the last CTA's staged rows and the splits' weights fit in the rings,
-  // and the ticket words fit their region.
-  // Measured on B200: it pays for the two-tile kernel (256 rows per CTA: the merge kernel re-reads
-  // large partials from DRAM after the grid ends), not for one-tile CTAs (many short CTAs pay the
-  // fence and ticket round trips; many splits leave one CTA a long merge), which keep the merge
-  // kernel.  TSD_ATTN_MERGE=kernel / =fused force either choice (A/B runs).
-  const char* merge_env = getenv("TSD_ATTN_MERGE");
-  const long long groups = (long long)a.B * a.Hkv * u.mtiles;
-  const bool want = merge_env != nullptr ? merge_env[0] == 'f' : p.dual;
-  const bool fuse = want && tickets != nullptr && u.splits > 1 && u.stage &&
-                    (size_t)(u.ks + u.vs) * kSlot >= (size_t)rows * kStageF + (size_t)u.splits * rows * 12 &&
-                    groups * 4 <= (long long)kAttnTicketBytes;
+  UmmaLayout L;
+  if (!umma_layout(p, G, a.Nmax, L)) return TSD_ERR_INVALID_ARG;
+  u.W = L.W, u.ks = L.ks, u.vs = L.vs, u.stage = L.stage;
+  u.k_off = L.k_off, u.v_off = L.v_off, u.mask_off = L.mask_off, u.ps_off = L.ps_off;
+  const bool fuse = tickets != nullptr && umma_merges_in_kernel(p, L, a.B, a.Hkv);
   u.tickets = fuse ? tickets : nullptr;
   *merged = fuse;
-  const size_t smem = total(u.ks, u.vs);
+  const size_t smem = L.smem;
 
   CUtensorMap mq, mk, mv, mkt, mvt;
   {  // Q [B*Nmax rows][Hq][128] -> box (64, G, 128/G)

@@ -97,6 +97,19 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
 tsd_status launch_attention(const AttnArgs& a, tsd_dtype dtype, cudaStream_t stream);
 // tcgen05 path (attn_umma.cu): bf16, d = 128, tree K/V in their own buffer, G a power of two.
 bool umma_eligible(const AttnArgs& a, tsd_dtype dtype);
+// Shared-memory layout of one tcgen05 attention CTA (rings, staged epilogue rows).
+struct UmmaLayout {
+  int rows = 0, W = 0, ks = 0, vs = 0, stage = 0;
+  uint32_t k_off = 0, v_off = 0, mask_off = 0, ps_off = 0;
+  size_t smem = 0;
+};
+bool umma_layout(const AttnPlan& p, int G, int Nmax, UmmaLayout& L);
+bool umma_merges_in_kernel(const AttnPlan& p, const UmmaLayout& L, int B, int Hkv);
+// Kernels one attention call launches (split kernel, plus the merge kernel when the keys are split
+// and not merged in the kernel), for 16-byte-aligned tensors and a workspace of the queried size.
+int attention_launch_count(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype, bool paged,
+                           bool tree_in_cache);
+
 // `tickets` (may be null) enables the split merge inside the kernel; *merged says whether it ran
 // there (otherwise the caller launches the merge kernel).
 tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, int* tickets, bool* merged,

@@ -31,8 +31,9 @@ from typing import Optional
 import torch
 
 from . import (tree_prepare, tree_verify_attn, tree_verify_attn_paged, tree_accept_greedy, chain_accept_sample,
-               kv_commit, kv_commit_paged, tree_accept_commit, tree_verify_attn_workspace_size, tree_verify_attn_paged_workspace_size,
-               tree_accept_greedy_workspace_size, chain_accept_sample_workspace_size, TSD_BF16, TSD_F32)
+               kv_commit, kv_commit_paged, tree_accept_commit, tree_verify_attn_workspace_size,
+               tree_verify_attn_paged_workspace_size, tree_verify_attn_kernels, tree_accept_greedy_workspace_size,
+               chain_accept_sample_workspace_size, TSD_BF16, TSD_F32)
 
 
 class VerifyStep:
@@ -80,7 +81,10 @@ class VerifyStep:
             self.out_tokens = torch.zeros(B, K + 1, **i32)
         self.history = torch.zeros(B, history_cap, **i32) if history_cap > 0 and self.fused else None
         self.history_len = torch.zeros(B, **i32) if self.history is not None else None
-        self.splits_merge = ws > 0   # the plan splits the keys: a merge launch follows the attention
+        # kernels of one attention call: the split kernel, and a merge kernel when the keys are split
+        # and not merged inside it
+        cap = max_blocks * block_size if paged else Lmax
+        self.attn_kernels = tree_verify_attn_kernels(B, Nmax, Hq, Hkv, d, cap, dt, block_size if paged else 0)
         if schedule == "overlap":
             self.side = torch.cuda.Stream(device=dev)
             self.ev_fork, self.ev_join = torch.cuda.Event(), torch.cuda.Event()
@@ -88,14 +92,14 @@ class VerifyStep:
     def launches_per_step(self) -> int:
         """Kernels one run() launches: prepare, attention (+ split merge), acceptance (scan +
         decide, or the chain sampler's three), commit (inside the fused acceptance)."""
-        n = 2 + int(self.splits_merge)
+        n = 1 + self.attn_kernels
         if self.accept == "greedy":
             return n + (2 if self.fused else 3)
         return n + (4 if self.T > 0 else 2) + 1
 
     def attn_launches(self) -> int:
         """Kernels one attention call launches (the split kernel, and its merge when split)."""
-        return 1 + int(self.splits_merge)
+        return self.attn_kernels
 
     def _accept(self, x: dict):
         if self.accept == "greedy":
