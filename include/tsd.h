@@ -57,6 +57,12 @@
  *     outputs are zero-filled where the call has outputs).  An error a call detects itself is
  *     stored into status[b] only if status[b] is still 0 (the first error wins); that
  *     sequence's outputs of that call are then zero-filled.
+ *   - Environment knobs of the attention, read at each call (A/B runs and tests; the defaults
+ *     are the measured choices): TSD_ATTN_PATH=mma (the warp-level mma.sync kernel where the
+ *     tcgen05 kernel applies), TSD_ATTN_DUAL=0 (one query tile per CTA), TSD_ATTN_SPLITS=n (the
+ *     tcgen05 kernel's key splits, when the workspace holds n partials), TSD_ATTN_MERGE=kernel|fused
+ *     (where the splits are merged), TSD_TEST_WITHHOLD_TILE=t (test hook: the K producer skips
+ *     key tile t and the bounded waits give up after 1e5 cycles, reporting TSD_ERR_TIMEOUT).
  */
 #ifndef TSD_H_
 #define TSD_H_
