@@ -61,7 +61,8 @@
  *     are the measured choices): TSD_ATTN_PATH=mma (the warp-level mma.sync kernel where the
  *     tcgen05 kernel applies), TSD_ATTN_DUAL=0 (one query tile per CTA), TSD_ATTN_SPLITS=n (the
  *     tcgen05 kernel's key splits, when the workspace holds n partials), TSD_ATTN_MERGE=kernel|fused
- *     (where the splits are merged), TSD_TEST_WITHHOLD_TILE=t (test hook: the K producer skips
+ *     (where the splits are merged), TSD_ATTN_L2HINT=0 (no evict-first L2 policy on K/V tiles read
+ *     once), TSD_TEST_WITHHOLD_TILE=t (test hook: the K producer skips
  *     key tile t and the bounded waits give up after 1e5 cycles, reporting TSD_ERR_TIMEOUT).
  */
 #ifndef TSD_H_

@@ -84,6 +84,7 @@ struct UParams {
   int W;               // ancestor-bit words per node
   int stage;           // epilogue rows go through shared memory (the ring region is large enough)
   int* tickets;        // split merge in the kernel: one ticket word per row block (null: merge kernel)
+  int evict_first;     // the cache's K/V tiles are read once: load them with an evict-first L2 policy
   uint32_t k_off, v_off, mask_off, ps_off;   // shared-memory offsets
 };
 
@@ -164,13 +165,16 @@ __device__ __forceinline__ void fetch_blocks(const AttnArgs& a, const SeqView& v
 __device__ __forceinline__ void load_tile(const AttnArgs& a, const SeqView& v, const UParams& u, int b, int g,
                                           int t, uint8_t* dst, const CUtensorMap* cache_map,
                                           const CUtensorMap* tree_map, uint64_t* bar, int* s_err,
-                                          const TileBlocks& tb) {
+                                          const TileBlocks& tb, uint64_t pol) {
+  // cache tiles go in under the producer's L2 policy: evict-first when the whole grid reads each
+  // tile once (the split partials written meanwhile then stay in L2 for the merge)
+  auto load2 = [&](uint8_t* d, int x, int y) { tma_load_2d_hint(d, cache_map, x, y, bar, pol); };
   if (t < v.nPT) {
     const int pos0 = t * kBN;
     if (a.block_table == nullptr) {
       const int y = (b * a.Hkv + g) * a.Lcap + pos0;
-      tma_load_2d(dst, cache_map, 0, y, bar);
-      tma_load_2d(dst + kHalf, cache_map, 64, y, bar);
+      load2(dst, 0, y);
+      load2(dst + kHalf, 64, y);
     } else {
       const int bs_mask = (1 << a.block_shift) - 1;
 #pragma unroll
@@ -185,8 +189,8 @@ __device__ __forceinline__ void load_tile(const AttnArgs& a, const SeqView& v, c
         }
         const int y = (blk * a.Hkv + g) * (1 << a.block_shift) + (pos & bs_mask);
         const uint32_t off = (uint32_t)seg * 128;
-        tma_load_2d(dst + off, cache_map, 0, y, bar);
-        tma_load_2d(dst + kHalf + off, cache_map, 64, y, bar);
+        load2(dst + off, 0, y);
+        load2(dst + kHalf + off, 64, y);
       }
     }
   } else {
@@ -469,6 +473,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         tma_load_3d(sQ + kQBytes / 2, &tmQ, 64, g * G, zq, &bars.q_full);
       }
       int issued = 0;
+      const uint64_t pol = u.evict_first ? l2_evict_first_policy() : l2_evict_normal_policy();
       TileBlocks nxt;
       fetch_blocks(a, v, u, b, t_begin, nxt);
       for (int i = 0; i < nt && !s_abort; ++i) {
@@ -481,7 +486,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           break;
         }
         mbar_expect_tx(&bars.k_full[st], kSlot);
-        load_tile(a, v, u, b, g, t_begin + i, sK + (size_t)st * kSlot, &tmK, &tmKt, &bars.k_full[st], &s_err, cur);
+        load_tile(a, v, u, b, g, t_begin + i, sK + (size_t)st * kSlot, &tmK, &tmKt, &bars.k_full[st], &s_err, cur,
+                  pol);
         ++issued;
       }
       s_k_issued = issued;
@@ -499,6 +505,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     // ------------------------------------------------------------ V producer (one thread)
     if (lane == 0) {
       int issued = 0;
+      const uint64_t pol = u.evict_first ? l2_evict_first_policy() : l2_evict_normal_policy();
       TileBlocks nxt;
       fetch_blocks(a, v, u, b, t_begin, nxt);
       for (int i = 0; i < nt && !s_abort; ++i) {
@@ -510,7 +517,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           break;
         }
         mbar_expect_tx(&bars.v_full[st], kSlot);
-        load_tile(a, v, u, b, g, t_begin + i, sV + (size_t)st * kSlot, &tmV, &tmVt, &bars.v_full[st], &s_err, cur);
+        load_tile(a, v, u, b, g, t_begin + i, sV + (size_t)st * kSlot, &tmV, &tmVt, &bars.v_full[st], &s_err, cur,
+                  pol);
         ++issued;
       }
       s_v_issued = issued;
@@ -1056,6 +1064,10 @@ tsd_status launch_attention_umma(const AttnArgs& a, const AttnPlan& p, int* tick
   u.wait = kWaitCycles;
   u.withhold = -1;
   u.lpt = a.B > 1 && a.B <= kThreadsU ? 1 : 0;
+  // one row block per KV head: every cache tile is read once by the whole grid (TSD_ATTN_L2HINT=0
+  // turns the evict-first policy off, for A/B runs)
+  const char* l2_env = getenv("TSD_ATTN_L2HINT");
+  u.evict_first = (p.umtiles == 1 && !(l2_env != nullptr && l2_env[0] == '0')) ? 1 : 0;
   // Test hook for the bounded waits: TSD_TEST_WITHHOLD_TILE=t makes the K producer of every CTA
   // skip key tile t (and every later one), so the waits on it give up after 10^5 cycles and the
   // call reports TSD_ERR_TIMEOUT in status[] instead of stalling.
