@@ -183,6 +183,12 @@ size_t tsd_tree_verify_attn_ticket_bytes(void);
 int tsd_tree_verify_attn_kernels(int B, int Nmax, int Hq, int Hkv, int d, int Lmax, int block_size, int tree_in_cache,
                                  tsd_dtype dtype);
 
+/* CTAs of the attention call's split kernel for the same arguments (its grid: a caller that runs
+ * other work beside the attention can tell whether the grid alone fills the GPU).  0 for invalid
+ * sizes. */
+long long tsd_tree_verify_attn_ctas(int B, int Nmax, int Hq, int Hkv, int d, int Lmax, int block_size,
+                                    int tree_in_cache, tsd_dtype dtype);
+
 tsd_status tsd_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache, int Lmax,
                                 const int32_t *prefix_len, const void *k_tree, const void *v_tree,
                                 const int32_t *parent_s, const int32_t *num_nodes, int B, int Nmax, int Hq,

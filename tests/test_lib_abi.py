@@ -159,3 +159,14 @@ def test_attention_kernel_count_query(monkeypatch):
     monkeypatch.setenv("TSD_ATTN_MERGE", "fused")
     assert q(1, 26, 32, 8, 128, 2112, 1) == 1
     assert q(0, 26, 32, 8, 128, 2112, 1) == 0
+
+
+def test_attention_grid_query():
+    """CTAs of the split kernel for the bench shapes (B x KV heads x row blocks x key splits): the
+    step launches an attention grid smaller than the GPU before the acceptance, a larger one after."""
+    q = tsd.tree_verify_attn_ctas
+    assert q(1, 26, 32, 8, 128, 2112, 1) == 1 * 8 * 1 * 9           # tree26
+    assert q(16, 60, 32, 8, 128, 520 * 16, 1, 16) == 16 * 8 * 1 * 2  # eagle60: two query tiles per CTA
+    assert q(64, 6, 64, 8, 128, 8256, 1) == 64 * 8 * 1 * 2           # chain5
+    assert q(8, 512, 32, 8, 128, 2080 * 16, 1, 16) == 8 * 8 * 8 * 2  # forest: 8 row blocks of 256 rows
+    assert q(0, 26, 32, 8, 128, 2112, 1) == 0

@@ -41,6 +41,7 @@ _SIGS = {
     "tsd_tree_verify_attn_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "tsd_tree_verify_attn_ticket_bytes": (_SZ, []),
     "tsd_tree_verify_attn_kernels": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "tsd_tree_verify_attn_ctas": (C.c_longlong, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "tsd_tree_verify_attn_paged": (_I, [_P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                         _I, _F, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_accept_greedy_workspace_size": (_SZ, [_I, _I, _I]),
@@ -176,6 +177,11 @@ def tree_verify_attn_kernels(B, Nmax, Hq, Hkv, d, Lmax, dtype, block_size: int =
     """Kernels one attention call launches for these sizes (the split kernel, and the merge kernel
     when the keys are split and not merged inside it); Lmax = capacity, block_size 0 = contiguous."""
     return int(lib().tsd_tree_verify_attn_kernels(B, Nmax, Hq, Hkv, d, Lmax, block_size, int(tree_in_cache), dtype))
+
+
+def tree_verify_attn_ctas(B, Nmax, Hq, Hkv, d, Lmax, dtype, block_size: int = 0, tree_in_cache: bool = False) -> int:
+    """CTAs of the attention call's split kernel for these sizes (its grid)."""
+    return int(lib().tsd_tree_verify_attn_ctas(B, Nmax, Hq, Hkv, d, Lmax, block_size, int(tree_in_cache), dtype))
 
 
 def _nbytes(ws) -> int:

@@ -81,6 +81,14 @@ int tsd_tree_verify_attn_kernels(int B, int Nmax, int Hq, int Hkv, int d, int Lm
   return attention_launch_count(B, Nmax, Hq, Hkv, d, Lmax, dtype, block_size > 0, tree_in_cache != 0);
 }
 
+long long tsd_tree_verify_attn_ctas(int B, int Nmax, int Hq, int Hkv, int d, int Lmax, int block_size,
+                                    int tree_in_cache, tsd_dtype dtype) {
+  if (B <= 0 || Nmax <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Lmax < 0 || block_size < 0 || !dtype_ok(dtype)) return 0;
+  long long n = 0;
+  attention_launch_count(B, Nmax, Hq, Hkv, d, Lmax, dtype, block_size > 0, tree_in_cache != 0, &n);
+  return n;
+}
+
 size_t tsd_tree_verify_attn_paged_workspace_size(int B, int Nmax, int Hq, int Hkv, int d, int max_blocks,
                                                  int block_size, tsd_dtype dtype) {
   if (max_blocks < 0 || block_size <= 0) return 0;

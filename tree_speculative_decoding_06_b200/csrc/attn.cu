@@ -624,7 +624,8 @@ AttnPlan plan_attention(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_d
 }
 
 int attention_launch_count(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype, bool paged,
-                           bool tree_in_cache) {
+                           bool tree_in_cache, long long* ctas) {
+  if (ctas) *ctas = 0;
   if (B <= 0 || Nmax <= 0 || Hkv <= 0) return 0;
   const AttnPlan p = plan_attention(B, Nmax, Hq, Hkv, d, Lcap, dtype, paged);
   const char* path_env = getenv("TSD_ATTN_PATH");
@@ -633,6 +634,9 @@ int attention_launch_count(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, ts
   // the tcgen05 kernel's conditions (umma_eligible), for aligned tensors
   const bool umma = dtype == TSD_BF16 && d == 128 && !tree_in_cache && G >= 1 && G <= 128 && (G & (G - 1)) == 0 &&
                     Lcap > 0 && !force_mma;
+  if (ctas) {
+    *ctas = umma ? (long long)B * Hkv * p.umtiles * p.usplits : (long long)B * Hkv * p.mtiles * p.splits;
+  }
   if (!umma) return p.splits > 1 ? 2 : 1;
   if (p.usplits <= 1) return 1;
   UmmaLayout L;

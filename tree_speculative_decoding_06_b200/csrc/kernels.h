@@ -107,8 +107,9 @@ bool umma_layout(const AttnPlan& p, int G, int Nmax, UmmaLayout& L);
 bool umma_merges_in_kernel(const AttnPlan& p, const UmmaLayout& L, int B, int Hkv);
 // Kernels one attention call launches (split kernel, plus the merge kernel when the keys are split
 // and not merged in the kernel), for 16-byte-aligned tensors and a workspace of the queried size.
+// (*ctas, if given: the CTAs of the split kernel's grid.)
 int attention_launch_count(int B, int Nmax, int Hq, int Hkv, int d, int Lcap, tsd_dtype dtype, bool paged,
-                           bool tree_in_cache);
+                           bool tree_in_cache, long long* ctas = nullptr);
 
 // `tickets` (may be null) enables the split merge inside the kernel; *merged says whether it ran
 // there (otherwise the caller launches the merge kernel).
