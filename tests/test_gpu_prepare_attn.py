@@ -222,3 +222,27 @@ def test_merge_tickets_return_to_zero_and_garbage_is_reported(name, monkeypatch)
     out, lse, st = gpu_attention(inp, workspace=ws)
     assert (st == 0).all()
     check_attention(inp, out, lse)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_merge_in_kernel_with_flagged_sequences(paged, monkeypatch):
+    """The in-kernel split merge on the sequences a call must zero: one whose tree prepare flags on
+    entry (a malformed parent) and one past the cache capacity.  Every CTA of such a row block
+    leaves early but still takes its ticket, the last one zeroes the rows, the ticket words return
+    to zero, and the other sequences are exact (two query tiles per CTA: 26 nodes x 8 heads)."""
+    monkeypatch.setenv("TSD_ATTN_SPLITS", "3")
+    monkeypatch.setenv("TSD_ATTN_MERGE", "fused")
+    tree = W.tree_static_scored((4, 3, 2, 1, 1, 1), 26)
+    inp = W.make_custom_inputs([tree] * 4, [300, 500, 200, 420], Hq=32, Hkv=4, d=128, dtype="bf16", seed=9,
+                               paged=paged)
+    inp["parent"] = inp["parent"].copy()
+    inp["parent"][1, 5] = 9                               # a forward parent: prepare flags sequence 1
+    inp["prefix_len"] = inp["prefix_len"].copy()
+    inp["prefix_len"][2] = inp["Lmax"] + 1                # past the capacity: the attention flags sequence 2
+    ws = forced_split_workspace(inp)
+    for _ in range(2):
+        out, lse, st = gpu_attention(inp, workspace=ws)
+        assert st[0] == 0 and st[3] == 0 and (st[1] & 0xFF) == 3 and (st[2] & 0xFF) == 6, st
+        assert (out[1] == 0).all() and (out[2] == 0).all()
+        assert int(_ticket_words(ws).abs().sum()) == 0
+    check_attention(inp, out, lse, rows=[(b, i, h) for b in (0, 3) for i in range(26) for h in range(0, 32, 5)])
