@@ -102,7 +102,8 @@ typedef enum tsd_commit_mode {
 /* Name of a status code (a static string). */
 const char *tsd_status_str(int code);
 
-/* ABI version of this header (bumped on any signature change). */
+/* ABI version of this header (bumped on any signature or contract change; 2: the attention
+ * workspace starts with split-merge ticket words that must be zero before its first use). */
 int tsd_abi_version(void);
 
 /* ---------------------------------------------------------------------------------------

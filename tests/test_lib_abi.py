@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert tsd.lib().tsd_abi_version() == 1
+    assert tsd.lib().tsd_abi_version() == 2
     for code, name in tsd.STATUS.items():
         assert tsd.status_str(code) == name
     assert tsd.status_str(3 | (17 << 8)) == "TSD_ERR_BAD_TREE"

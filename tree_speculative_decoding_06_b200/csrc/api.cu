@@ -10,7 +10,7 @@ using namespace tsd;
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
